@@ -1,0 +1,284 @@
+"""CPU oracle for one Wave Forcing wave round -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference legs may import or run this module.  The product path (the CUDA
+library and its binding) never calls it, and it shares no code with that path.
+
+Plain, slow, obviously-correct NumPy in fp64 with an explicit visibility mask.
+What it follows:
+
+* Chunk-wise causal attention over earlier, cleaner chunks whose denoising is
+  not finished ("Wave Forcing: Towards Speed-of-Light Streaming Video
+  Generation", arXiv 2611.00859v1, Abstract), i.e. a new chunk conditions on a
+  mixed-noise frontier and not only on a clean prior chunk ("Wave Forcing from
+  SJTU-DENG Lab: 8 GPUs can't fix a missing sgl-dlab package", first
+  paragraph).
+* KV-cached chunk-autoregressive generation where the finished chunk's K/V are
+  written into the cache ("scope-causal-forcing", "How It Works", steps 1-2);
+  the denoising list [1000, 750, 500, 250] ("scope-causal-forcing",
+  "Configuration" table) supplies the in-round noise levels.
+
+Readings where the pages are silent (each is a parameter or a stated choice):
+
+* Mask: chunk i sees every cache chunk, the in-round chunks j <= i and all of
+  its own tokens (bidirectional inside a chunk); all in-round chunks share the
+  same cache window.
+* Age order: in-round index 0 is the oldest and cleanest chunk; noise levels
+  are metadata that never enter the attention arithmetic.
+* 3D RoPE (not on the pages): textbook rotary embedding (Su et al., RoFormer,
+  2021) applied per axis to interleaved (even, odd) pairs; pairs split into
+  consecutive groups P_t | P_h | P_w; frequency of pair k in a group of P pairs
+  is theta^(-k/P); positions are absolute from stream start (t = n*F + f).
+  Default split: P_h = P_w = floor((D/2)/3), P_t = D/2 - 2*P_h.
+* Ring: slot(n) = n mod S over S pool slots; the cache holds the last Wc
+  chunks before the round's oldest in-round chunk n0.
+* Scale 1/sqrt(D); rotated Q/K rounded to the storage type (nearest, ties to
+  even) from the fp64 rotation; attention itself in fp64.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+KEY_TILE = 128
+Q_TILE = 128
+Q_PAIR = 256
+
+
+# --------------------------------------------------------------------------
+# rounding to the storage types
+# --------------------------------------------------------------------------
+
+def round_bf16(x) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), kept in fp64.
+
+    bf16 keeps 8 significant bits and the fp32 exponent range: for
+    x = m * 2^e (0.5 <= |m| < 1) the spacing of bf16 values is 2^(e-8) for
+    normal results and the fixed subnormal spacing 2^-133 below 2^-126.
+    Scaling by a power of two and np.rint (ties to even) are exact.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    q_exp = np.maximum(e.astype(np.int64) - 8, -133)
+    q = np.ldexp(x, -q_exp)
+    r = np.ldexp(np.rint(q), q_exp)
+    big = np.abs(r) > 3.3895313892515355e38  # largest finite bf16
+    return np.where(big, np.copysign(np.inf, x), r)
+
+
+def round_f32(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def round_to(x, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return round_bf16(x)
+    if dtype == "f32":
+        return round_f32(x)
+    raise ValueError(dtype)
+
+
+# --------------------------------------------------------------------------
+# token geometry and 3D RoPE
+# --------------------------------------------------------------------------
+
+def chunk_len(F: int, fh: int, fw: int) -> int:
+    return F * fh * fw
+
+
+def token_positions(n: int, F: int, fh: int, fw: int):
+    """(t, h, w) of every token of global chunk n; tokens are (frame, row, col)."""
+    j = np.arange(F * fh * fw)
+    f = j // (fh * fw)
+    l = j % (fh * fw)
+    return n * F + f, l // fw, l % fw
+
+
+def rope_split(D: int):
+    ph = (D // 2) // 3
+    return D // 2 - 2 * ph, ph, ph
+
+
+def rope_angles(t, h, w, pairs, theta: float) -> np.ndarray:
+    """Angles [tokens, D/2]: each axis' positions times theta^(-k/P) for its group."""
+    cols = []
+    for pos, P in zip((t, h, w), pairs):
+        if P == 0:
+            continue
+        k = np.arange(P)
+        freq = np.float64(theta) ** (-k / P)
+        cols.append(np.asarray(pos, dtype=np.float64)[:, None] * freq[None, :])
+    return np.concatenate(cols, axis=1)
+
+
+def rope_rotate(x, angles) -> np.ndarray:
+    """Rotate interleaved pairs of x [tokens, ..., D] by angles [tokens, D/2] (fp64)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = angles.reshape(angles.shape[0], *([1] * (x.ndim - 2)), angles.shape[1])
+    c, s = np.cos(a), np.sin(a)
+    ev, od = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = ev * c - od * s
+    out[..., 1::2] = ev * s + od * c
+    return out
+
+
+def rope3d_chunk(x, n: int, F: int, fh: int, fw: int, pairs, theta: float) -> np.ndarray:
+    """Exact (fp64) 3D RoPE of chunk n's tensor x [C, H, D]."""
+    t, h, w = token_positions(n, F, fh, fw)
+    return rope_rotate(x, rope_angles(t, h, w, pairs, theta))
+
+
+# --------------------------------------------------------------------------
+# ring cache
+# --------------------------------------------------------------------------
+
+def ring_slot(n: int, S: int) -> int:
+    return n % S
+
+
+def cache_window(n0: int, Wc: int):
+    """Global indices of the clean cache chunks seen by the round starting at n0."""
+    return list(range(max(0, n0 - Wc), n0))
+
+
+def ring_contents_after(appends, S: int):
+    """Simulate appends of global chunk ids into an S-slot ring; slot -> chunk id."""
+    slots = [None] * S
+    for n in appends:
+        slots[ring_slot(n, S)] = n
+    return slots
+
+
+# --------------------------------------------------------------------------
+# plan re-derivation (visibility, slots, segments, work list)
+# --------------------------------------------------------------------------
+
+def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas):
+    """Re-derive the round plan: per-chunk visibility/slots and the LPT work list."""
+    C = F * fh * fw
+    wc_eff = min(Wc, n0)
+    first = n0 - wc_eff
+    chunks = []
+    for i in range(R):
+        n = n0 + i
+        nvis = wc_eff + i + 1
+        vis = [first + k for k in range(nvis)]
+        s0 = first % S
+        len0 = min(nvis, S - s0)
+        segs = [(s0 * C, len0 * C), (0, (nvis - len0) * C)]
+        tiles = sum(-(-ln // KEY_TILE) for _, ln in segs)
+        chunks.append(dict(n=n, slot=n % S, noise=int(noise_t[i]), nvis=nvis,
+                           vis_chunks=vis, vis_slots=[v % S for v in vis],
+                           keys=nvis * C, segs=segs, key_tiles=tiles))
+    pairs = -(-C // Q_PAIR)
+    units = []
+    for i in range(R):
+        for h in range(H):
+            for p in range(pairs):
+                rows = min(Q_PAIR, C - Q_PAIR * p)
+                live = 1 if rows <= Q_TILE else 2
+                units.append((i, h, p, chunks[i]["key_tiles"] * live))
+    units.sort(key=lambda u: (-u[3], -u[0], u[1], u[2]))
+    loads = [0] * num_ctas
+    per_cta = [[] for _ in range(num_ctas)]
+    for u in units:
+        c = min(range(num_ctas), key=lambda k: (loads[k], k))
+        per_cta[c].append(u)
+        loads[c] += u[3]
+    return dict(C=C, wc_eff=wc_eff, first=first, chunks=chunks, units=units,
+                per_cta=per_cta, loads=loads, q_pairs=pairs)
+
+
+# --------------------------------------------------------------------------
+# visibility mask and attention
+# --------------------------------------------------------------------------
+
+def logical_key_chunks(wc_eff: int, R: int):
+    """Logical key order: cache chunks (oldest first) then in-round chunks 0..R-1.
+    Returns (is_cache, in-round index or -1) per key chunk."""
+    return [(True, -1)] * wc_eff + [(False, i) for i in range(R)]
+
+
+def visibility_mask(C: int, wc_eff: int, R: int, q_chunks=None) -> np.ndarray:
+    """M[q, k] = 1 iff key chunk is cache or an in-round chunk j <= query chunk i."""
+    q_chunk = np.repeat(np.arange(R), C) if q_chunks is None else np.asarray(q_chunks)
+    kinfo = logical_key_chunks(wc_eff, R)
+    k_is_cache = np.repeat(np.array([c for c, _ in kinfo], dtype=bool), C)
+    k_chunk = np.repeat(np.array([i for _, i in kinfo]), C)
+    return k_is_cache[None, :] | (k_chunk[None, :] <= q_chunk[:, None])
+
+
+def attention(q, k, v, mask, scale: float):
+    """softmax(q k^T * scale, masked) v in fp64; q [nq,D], k/v [nk,D], mask [nq,nk].
+    Returns (O [nq,D], LSE [nq]) with LSE = log sum_k exp(scale * q.k) over visible keys."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    s = (q @ k.T) * scale
+    s = np.where(mask, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p @ v) / l, (m + np.log(l))[:, 0]
+
+
+def attention_bruteforce(q, k, v, mask, scale: float):
+    """Per-query Python loop over visible keys, no max subtraction (tiny inputs only)."""
+    nq, D = len(q), len(q[0])
+    out = np.zeros((nq, D))
+    lse = np.zeros(nq)
+    for a in range(nq):
+        num = [0.0] * D
+        den = 0.0
+        for b in range(len(k)):
+            if not mask[a][b]:
+                continue
+            dot = 0.0
+            for d in range(D):
+                dot += float(q[a][d]) * float(k[b][d])
+            w = math.exp(dot * scale)
+            den += w
+            for d in range(D):
+                num[d] += w * float(v[b][d])
+        out[a] = [x / den for x in num]
+        lse[a] = math.log(den)
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# one wave round
+# --------------------------------------------------------------------------
+
+def wave_round(q_raw, k_raw, v_raw, k_cache_raw, v_cache_raw, *, n0, F, fh, fw,
+               pairs, theta, dtype, scale=None, rows=None):
+    """One wave round for the heads present in the inputs.
+
+    q_raw/k_raw/v_raw: [R, C, H, D] raw in-round tensors (chunk i is global n0+i);
+    k_cache_raw/v_cache_raw: [Wc_eff, C, H, D] raw K/V of cache chunks
+    n0-Wc_eff .. n0-1 as they were when last appended.
+    rows: optional in-round query indices (flat over R*C) to evaluate.
+    Returns dict with q_rot [R,C,H,D], k_rot [R,C,H,D], k_cache_rot, O [nrows,H,D],
+    LSE [nrows,H] -- rotated tensors rounded to ``dtype``.
+    """
+    R, C, H, D = q_raw.shape
+    wc_eff = k_cache_raw.shape[0]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rot = lambda x, n: round_to(rope3d_chunk(x, n, F, fh, fw, pairs, theta), dtype)
+    q_rot = np.stack([rot(q_raw[i], n0 + i) for i in range(R)])
+    k_rot = np.stack([rot(k_raw[i], n0 + i) for i in range(R)])
+    kc_rot = (np.stack([rot(k_cache_raw[c], n0 - wc_eff + c) for c in range(wc_eff)])
+              if wc_eff else np.zeros((0, C, H, D)))
+    vr = round_to(v_raw, dtype)
+    vc = round_to(v_cache_raw, dtype) if wc_eff else np.zeros((0, C, H, D))
+    keys = np.concatenate([kc_rot, k_rot]).reshape(-1, H, D)
+    vals = np.concatenate([vc, vr]).reshape(-1, H, D)
+    rows = np.arange(R * C) if rows is None else np.asarray(rows)
+    mask = visibility_mask(C, wc_eff, R, q_chunks=rows // C)
+    qf = q_rot.reshape(-1, H, D)[rows]
+    out = np.zeros((len(rows), H, D))
+    lse = np.zeros((len(rows), H))
+    for h in range(H):
+        out[:, h], lse[:, h] = attention(qf[:, h], keys[:, h], vals[:, h], mask, scale)
+    return dict(q_rot=q_rot, k_rot=k_rot, k_cache_rot=kc_rot, v=vr, O=out, LSE=lse, rows=rows)
