@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the wave-round hot path on B200.
+
+A step is one wave round of a streaming rollout at the Wan2.1-1.3B shape
+(12 heads x 128, 30x52 tokens per frame, 3-frame chunks of 4680 tokens,
+7 cache chunks, 4 in-round chunks at staggered noise levels): host plan,
+RoPE/append of the round's new Q/K/V into the ring pool, and block-causal
+attention.  The ring advances one chunk per step.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU runs are independent replicas (the path has no exchange step): each
+rank runs its own rollout; the value is the work of all ranks divided by the
+slowest rank's device time.  The reference arm (--impl reference) times the
+CPU oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk-causal attn TFLOP/s & wave rounds/s at Wan-1.3B shape; % BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("wf", "reference"), default="wf")
+    ap.add_argument("--config", default="wan13b_round")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "wf_plan.h"):
+        with open(os.path.join(ROOT, "chunk_causal_attention_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(config):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
+    or None when the kernel source changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "attn_dram_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return t.get("bytes_per_launch", {}).get(config)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="wf_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        smax = max(float(r[2]) for r in rows)
+        loaded = [s for s, r in zip(sm, rows) if float(r[3]) > 200.0] or sm
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) sample
+
+def oracle_sample(cfg, seconds: float, first_n0: int, n0: int, seed: int = 42):
+    """Time the CPU oracle on a bounded sample of one round: whole heads, a
+    fixed set of query rows per chunk, every visible key (with its RoPE).
+    Returns (algorithmic flops done, seconds, description)."""
+    import numpy as np
+    from tests import gpu_common as gc
+
+    rows_per_chunk = 256
+    rows = np.concatenate([i * cfg.C + np.arange(rows_per_chunk) for i in range(cfg.R)])
+    flops_per_head = sum(4.0 * cfg.D * rows_per_chunk * k for k in cfg.visible_keys())
+    done, heads, t_total = 0.0, 0, 0.0
+    while t_total < seconds and heads < cfg.H:
+        arrays = gc.oracle_inputs(cfg, n0, first_n0, [heads], seed=seed)  # drawing is not timed
+        t0 = time.perf_counter()
+        gc.oracle_call(cfg, n0, arrays, rows=rows)
+        t_total += time.perf_counter() - t0
+        done += flops_per_head
+        heads += 1
+    desc = (f"oracle wave_round (fp64 NumPy) on {heads} head(s) x {rows_per_chunk} query rows per in-round "
+            f"chunk of round n0={n0}, all visible keys incl. their RoPE; input drawing excluded")
+    return done, t_total, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, rank, world):
+    """CPU oracle arm: rank 0 only, K timed steps of a bounded oracle sample."""
+    if rank != 0:
+        return None
+    import numpy as np  # noqa: F401
+    from chunk_causal_attention_block_b200.rollout import CONFIGS
+
+    cfg = CONFIGS[args.config]
+    # each step is a bounded sample (at least one head) so that the run stays within a few minutes
+    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup))
+    for w in range(args.warmup):
+        oracle_sample(cfg, 0.1, cfg.Wc, cfg.Wc + w)
+    flops, secs = 0.0, 0.0
+    desc = ""
+    for s in range(args.steps):
+        f, t, desc = oracle_sample(cfg, per_step, cfg.Wc, cfg.Wc + args.warmup + s)
+        flops += f
+        secs += t
+    value = flops / secs / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Irwin-Hall(12) N(0,1) draws, seed 42)",
+        "config": {"workload": cfg.name + " (oracle sample per step)", "heads": cfg.H, "head_dim": cfg.D,
+                   "chunk_tokens": cfg.C, "cache_chunks": cfg.Wc, "inround_chunks": cfg.R,
+                   "parallelism": f"replicas x{args.gpus} (reference arm runs on rank 0 only)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def run_wf(args, rank, world, local_rank):
+    import numpy as np  # noqa: F401
+    import torch
+    import torch.distributed as dist
+
+    from chunk_causal_attention_block_b200 import wf
+    from chunk_causal_attention_block_b200.rollout import CONFIGS, Rollout
+
+    wf.lib()  # fails loudly if the CUDA library is missing
+    cfg = CONFIGS[args.config]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    W, K = args.warmup, args.steps
+    ro = Rollout(cfg, device=dev, want_lse=False, seed=42 + rank)
+    ro.prefill()
+
+    # every step's inputs resident in HBM before timing (round r draws tag r)
+    tdt = torch.bfloat16 if cfg.dtype == wf.WF_BF16 else torch.float32
+    nq = cfg.R * cfg.C
+    inputs = []
+    for r in range(W + K):
+        q, k, v = (torch.empty(nq, cfg.H, cfg.D, dtype=tdt, device=dev) for _ in range(3))
+        for t, dst in ((wf.WF_SYNTH_Q, q), (wf.WF_SYNTH_K, k), (wf.WF_SYNTH_V, v)):
+            wf.wf_synth_fill(dst, cfg.dtype, ro.seed, t, r, ro.n0_of(r), cfg.R, cfg.C, cfg.H, cfg.D,
+                             kscale=(cfg.kscale and t == wf.WF_SYNTH_K), stream=stream)
+        inputs.append((q, k, v))
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    def step(r, events=None):
+        ro.q, ro.k, ro.v = inputs[r]
+        ro.plan_round(r)
+        if events:
+            events[0].record(stream)
+        ro.append()
+        if events:
+            events[1].record(stream)
+        ro.attend()
+        if events:
+            events[2].record(stream)
+
+    for r in range(W):
+        step(r)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(K):
+        step(W + s, ev[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end)
+    rope_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    code, detail = ro.device_status()
+    if code != wf.WF_OK:
+        raise RuntimeError(f"device status {wf.status_string(code)} {detail}")
+    ms_max = ms
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+
+    # end-to-end through the public calls with host buffers: H2D of the step's
+    # Q/K/V from pinned memory and D2H of O inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        nsets = min(4, W + K)
+        host_in = [tuple(x.cpu().pin_memory() for x in inputs[i]) for i in range(nsets)]
+        host_out = torch.empty(nq, cfg.H, cfg.D, dtype=tdt).pin_memory()
+        dq, dk, dv = (torch.empty_like(inputs[0][0]) for _ in range(3))
+        del inputs
+        torch.cuda.empty_cache()
+
+        def e2e_step(r):
+            hq, hk, hv = host_in[r % nsets]
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            ro.q, ro.k, ro.v = dq, dk, dv
+            ro.plan_round(r)
+            ro.append()
+            ro.attend()
+            host_out.copy_(ro.out[:nq], non_blocking=True)
+
+        base = W + K
+        for r in range(W):
+            e2e_step(base + r)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(K):
+            e2e_step(base + W + s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        elem = 2 if cfg.dtype == wf.WF_BF16 else 4
+        plan_bytes = ro.host_plan.numel()
+        e2e = {"value": cfg.attn_flops() * K * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 3 * nq * cfg.H * cfg.D * elem + plan_bytes,
+               "d2h_bytes_per_step": nq * cfg.H * cfg.D * elem,
+               "ms_per_step": e_ms / K}
+        code, detail = ro.device_status()
+        if code != wf.WF_OK:
+            raise RuntimeError(f"device status {wf.status_string(code)} {detail}")
+
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    flops = cfg.attn_flops()
+    attn_avg = statistics.mean(attn_ms)
+    rope_avg = statistics.mean(rope_ms)
+    achieved = flops / (attn_avg / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = dram_traffic(args.config)
+    value = flops * K * world / (ms_max / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == wf.WF_BF16 else "f32",
+        "data": "synthetic (seeded Irwin-Hall(12) N(0,1) draws, seed 42 + rank, drawn on device before timing)",
+        "config": {"workload": cfg.name, "heads": cfg.H, "head_dim": cfg.D,
+                   "tokens_per_frame": cfg.fh * cfg.fw, "chunk_tokens": cfg.C, "cache_chunks": cfg.Wc,
+                   "inround_chunks": cfg.R, "queries_per_round": nq,
+                   "visible_keys_per_chunk": cfg.visible_keys(), "global_batch": world,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (per-round Q/K/V 172 MB, K/V pool 316 MB, fresh inputs each step)"},
+        "wave_rounds_per_s": K * world / (ms_max / 1e3),
+        "attn_tflops_kernel": achieved,
+        "pct_bf16_peak": {"of_spec_2250": 100 * achieved / 2250.0,
+                          f"of_{peak_kind}_burst": 100 * achieved / peak,
+                          f"of_{peak_kind}_sustained": 100 * achieved / float(peaks["bf16_tflops_sustained"])},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "attn_fwd_sm100", "peak_kind": f"{peak_kind} bf16 burst"},
+        "rope_append": {"ms": rope_avg, "gb_s": cfg.rope_bytes() / (rope_avg / 1e3) / 1e9,
+                        "frac_of_hbm": cfg.rope_bytes() / (rope_avg / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+                        "bytes": cfg.rope_bytes()},
+        "attn_ms": attn_avg,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        f, t, desc = oracle_sample(cfg, args.cpu_seconds, ro.first_n0, ro.n0_of(0))
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc, "seconds": t}
+    return line
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the oracle arm is CPU-only; under torchrun only rank 0 works
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_wf(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

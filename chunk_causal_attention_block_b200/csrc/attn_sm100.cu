@@ -1,0 +1,525 @@
+// Block-causal flash-attention forward of one wave round on B200 tensor
+// cores (tcgen05 + TMEM + TMA), bf16 in/out, head_dim 128.
+//
+// Persistent kernel, one CTA per SM, each CTA working through the plan's
+// list of units (chunk i, head h, 256 query rows = two 128-row tiles).  The
+// visible keys of chunk i are the plan's one or two contiguous pool runs,
+// walked in 128-key tiles; tiles of chunks that chunk i may not see are never
+// loaded.  Only the last tile of a run can be ragged; its extra columns are
+// masked to -inf.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for query tile 0 (thread = one TMEM lane = one row)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    tcgen05.mma issue (lane 0) and TMEM allocation (whole warp)
+//   warp  9    TMA producer (lane 0)
+// TMEM (512 columns x 128 lanes x 32 bit):
+//   S_t = Q_t K^T at columns [128t, 128t+128), fp32; P_t (bf16 pairs) is
+//   written over the first 64 of them; O_t at [256+128t, 256+128t+128).
+// Shared memory: Q_0, Q_1 (32 KB each) and a ring of kStages 32 KB K/V tiles,
+// all 128-byte-swizzled, K-major for Q and K, MN-major for V.
+//
+// Per key tile j the MMA thread issues, in order,
+//   PV_0(j-1) .. S_0(j) .. PV_1(j-1) .. S_1(j)
+// so the commit that announces S_t(j) also covers PV_t(j-1): when a softmax
+// thread sees S_t(j) it owns O_t and may rescale it in place.  Online
+// softmax in the log2 domain with a lazily updated reference max: O is only
+// rescaled when a row's max grows by more than 8 (a factor 256), so P stays
+// below 256 and the fp32 sums stay exact enough; the final O / l uses the
+// same reference, so the result is unchanged.
+//
+// Every mbarrier wait is bounded by a time limit; on expiry the CTA records
+// WF_ERR_DEVICE_TIMEOUT in the workspace status word, stops issuing work,
+// drains what it issued and frees its TMEM before returning.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+#include "wf.h"
+#include "wf_plan.h"
+
+namespace wf {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
+constexpr int kHalfBytes = kTileBytes / 2; // one 64-column (128-byte) half
+constexpr int kSmemBytes = 1024 + 2 * kTileBytes + kStages * kTileBytes + 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);
+
+struct Params {
+  const wf_plan_chunk* chunks;
+  const wf_plan_unit* units;
+  const int32_t* cta_off;
+  __nv_bfloat16* out;
+  float* lse;
+  wf_dev_status* status;
+  int32_t H, C;
+  int32_t rc;            // R * C, the LSE row stride
+  float scale_log2;      // softmax scale * log2(e)
+  uint64_t timeout_ns;
+};
+
+// Barrier indices in the barrier block.
+enum : int {
+  kBarQFull = 0,
+  kBarQEmpty = 1,
+  kBarSFull = 2,     // +t
+  kBarPFull = 4,     // +t
+  kBarOFull = 6,     // +t
+  kBarMmaDone = 8,
+  kBarKVFull = 9,    // +stage
+  kBarKVEmpty = 9 + kStages,
+  kNumBars = 9 + 2 * kStages
+};
+
+struct Shared {
+  uint8_t* base;  // Q_0 | Q_1 | K/V stages, each kTileBytes, 1024-aligned
+  uint64_t* bars;
+  uint32_t* tmem_slot;
+  int32_t* abort_flag;
+};
+
+__device__ __forceinline__ uint8_t* q_tile(const Shared& s, int t) { return s.base + t * kTileBytes; }
+__device__ __forceinline__ uint8_t* kv_tile(const Shared& s, int st) { return s.base + (2 + st) * kTileBytes; }
+
+__device__ __forceinline__ Shared carve_smem(uint8_t* raw) {
+  Shared s;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.base = base;
+  uint8_t* tail = base + (2 + kStages) * kTileBytes;
+  s.bars = reinterpret_cast<uint64_t*>(tail);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(tail + 8 * kNumBars);
+  s.abort_flag = reinterpret_cast<int32_t*>(tail + 8 * kNumBars + 4);
+  return s;
+}
+
+// Bounded wait.  Returns false if this CTA is aborting (the wait expired here
+// or in another role); the first expiry records the status word.
+__device__ __forceinline__ bool wait_bar(const Shared& sh, const Params& p, int bar, uint32_t parity, int where) {
+  const uint32_t addr = smem_u32(sh.bars + bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(addr, parity)) return true;
+    if (*reinterpret_cast<volatile int32_t*>(sh.abort_flag)) return false;
+    if (global_timer_ns() - t0 > p.timeout_ns) {
+      *reinterpret_cast<volatile int32_t*>(sh.abort_flag) = 1;
+      if (atomicCAS(&p.status->code, 0, int32_t(WF_ERR_DEVICE_TIMEOUT)) == 0) {
+        p.status->where = where;
+        p.status->block = int32_t(blockIdx.x);
+        p.status->thread = int32_t(threadIdx.x);
+        __threadfence();
+      }
+      return false;
+    }
+  }
+}
+
+// Key tile j of chunk c: pool token of its first key and the number of valid keys.
+__device__ __forceinline__ void key_tile(const wf_plan_chunk& c, int j, int32_t& tok, int32_t& valid) {
+  // selects, not a dynamic index: keeps the record in registers
+  const bool first = j < c.seg_tiles[0];
+  const int t = first ? j : j - c.seg_tiles[0];
+  tok = (first ? c.seg_start[0] : c.seg_start[1]) + t * 128;
+  const int32_t left = (first ? c.seg_len[0] : c.seg_len[1]) - t * 128;
+  valid = left < 128 ? left : 128;
+}
+
+__device__ __forceinline__ wf_plan_chunk load_chunk(const wf_plan_chunk* p) {
+  wf_plan_chunk c;
+  c.seg_start[0] = __ldg(&p->seg_start[0]);
+  c.seg_start[1] = __ldg(&p->seg_start[1]);
+  c.seg_len[0] = __ldg(&p->seg_len[0]);
+  c.seg_len[1] = __ldg(&p->seg_len[1]);
+  c.seg_tiles[0] = __ldg(&p->seg_tiles[0]);
+  c.seg_tiles[1] = __ldg(&p->seg_tiles[1]);
+  c.key_tiles = __ldg(&p->key_tiles);
+  return c;
+}
+
+// ---------------------------------------------------------------- roles
+
+__device__ __forceinline__ void producer(const Shared& sh, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                         const CUtensorMap* tm_v, int u0, int u1) {
+  int kv_it = 0;
+  int q_it = 0;
+  bool ok = true;
+  for (int u = u0; u < u1 && ok; ++u) {
+    const wf_plan_unit unit = p.units[u];
+    const wf_plan_chunk c = load_chunk(p.chunks + unit.chunk);
+    const int32_t row0 = unit.chunk * p.C + unit.pair * 256;
+    const bool live1 = p.C - unit.pair * 256 > 128;
+    if (q_it > 0 && !wait_bar(sh, p, kBarQEmpty, (q_it - 1) & 1, 1)) { ok = false; break; }
+    const uint32_t qbar = smem_u32(sh.bars + kBarQFull);
+    mbar_arrive_expect_tx(qbar, live1 ? 2 * kTileBytes : kTileBytes);
+    tma_load_3d(smem_u32(q_tile(sh, 0)), tm_q, qbar, 0, unit.head, row0);
+    tma_load_3d(smem_u32(q_tile(sh, 0) + kHalfBytes), tm_q, qbar, 64, unit.head, row0);
+    if (live1) {
+      tma_load_3d(smem_u32(q_tile(sh, 1)), tm_q, qbar, 0, unit.head, row0 + 128);
+      tma_load_3d(smem_u32(q_tile(sh, 1) + kHalfBytes), tm_q, qbar, 64, unit.head, row0 + 128);
+    }
+    ++q_it;
+    for (int j = 0; j < c.key_tiles; ++j) {
+      int32_t tok, valid;
+      key_tile(c, j, tok, valid);
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const int st = kv_it % kStages;
+        if (!wait_bar(sh, p, kBarKVEmpty + st, ((kv_it / kStages) & 1) ^ 1, 2)) { ok = false; break; }
+        const uint32_t bar = smem_u32(sh.bars + kBarKVFull + st);
+        mbar_arrive_expect_tx(bar, kTileBytes);
+        const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
+        tma_load_3d(smem_u32(kv_tile(sh, st)), tm, bar, 0, unit.head, tok);
+        tma_load_3d(smem_u32(kv_tile(sh, st) + kHalfBytes), tm, bar, 64, unit.head, tok);
+        ++kv_it;
+      }
+      if (!ok) break;
+    }
+  }
+  // Drain: the CTA must not exit with bulk copies still landing in its smem.
+  if (!ok) {
+    for (int s = 0; s < kStages; ++s) {
+      if (kv_it <= s) continue;
+      const int last_fill = (kv_it - 1 - s) / kStages;  // fill count - 1 of stage s
+      const uint32_t addr = smem_u32(sh.bars + kBarKVFull + s);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(addr, uint32_t(last_fill) & 1) && global_timer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+    if (q_it > 0) {
+      const uint32_t addr = smem_u32(sh.bars + kBarQFull);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(addr, uint32_t(q_it - 1) & 1) && global_timer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void issue_s(uint32_t s_tmem, const uint8_t* q, const uint8_t* k) {
+  const uint32_t qa = smem_u32(q), ka = smem_u32(k);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    // K-major, 128-byte swizzle: 16-element K slices are 32 bytes apart
+    // inside a 64-element half; the second half starts 16 KB later.
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    mma_ss(s_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), kIdescQK,
+           kk > 0 ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, const uint8_t* v, bool accumulate) {
+  const uint32_t va = smem_u32(v);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    // V is MN-major (head_dim contiguous): 16 keys = 2 KB further on; the two
+    // 64-column halves are 16 KB apart (leading byte offset), 8-key groups
+    // 1 KB apart (stride byte offset).  P_t holds 2 bf16 per column.
+    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), kIdescPV,
+           (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, uint32_t tmem, int u0, int u1) {
+  int kv_it = 0, q_it = 0;
+  int p_cnt[2] = {0, 0};
+  bool ok = true;
+  const uint32_t s_tm[2] = {tmem + 0, tmem + 128};
+  const uint32_t o_tm[2] = {tmem + 256, tmem + 384};
+  for (int u = u0; u < u1 && ok; ++u) {
+    const wf_plan_unit unit = p.units[u];
+    const int n = __ldg(&p.chunks[unit.chunk].key_tiles);
+    const bool live1 = p.C - unit.pair * 256 > 128;
+    if (!wait_bar(sh, p, kBarQFull, q_it & 1, 10)) { ok = false; break; }
+    ++q_it;
+    tc_fence_after();
+    int kst = kv_it % kStages;
+    if (!wait_bar(sh, p, kBarKVFull + kst, (kv_it / kStages) & 1, 11)) { ok = false; break; }
+    ++kv_it;
+    tc_fence_after();
+    issue_s(s_tm[0], q_tile(sh, 0), kv_tile(sh, kst));
+    mma_commit(smem_u32(sh.bars + kBarSFull + 0));
+    if (live1) {
+      issue_s(s_tm[1], q_tile(sh, 1), kv_tile(sh, kst));
+      mma_commit(smem_u32(sh.bars + kBarSFull + 1));
+    }
+    mma_commit(smem_u32(sh.bars + kBarKVEmpty + kst));
+    if (n == 1) mma_commit(smem_u32(sh.bars + kBarQEmpty));
+    for (int j = 0; j < n; ++j) {
+      const int vst = kv_it % kStages;
+      if (!wait_bar(sh, p, kBarKVFull + vst, (kv_it / kStages) & 1, 12)) { ok = false; break; }
+      ++kv_it;
+      const bool more = j + 1 < n;
+      if (more) {
+        kst = kv_it % kStages;
+        if (!wait_bar(sh, p, kBarKVFull + kst, (kv_it / kStages) & 1, 13)) { ok = false; break; }
+        ++kv_it;
+      }
+      // tile 0
+      if (!wait_bar(sh, p, kBarPFull + 0, p_cnt[0] & 1, 14)) { ok = false; break; }
+      ++p_cnt[0];
+      tc_fence_after();
+      issue_pv(o_tm[0], s_tm[0], kv_tile(sh, vst), j > 0);
+      if (more) {
+        issue_s(s_tm[0], q_tile(sh, 0), kv_tile(sh, kst));
+        mma_commit(smem_u32(sh.bars + kBarSFull + 0));
+      } else {
+        mma_commit(smem_u32(sh.bars + kBarOFull + 0));
+      }
+      // tile 1
+      if (live1) {
+        if (!wait_bar(sh, p, kBarPFull + 1, p_cnt[1] & 1, 15)) { ok = false; break; }
+        ++p_cnt[1];
+        tc_fence_after();
+        issue_pv(o_tm[1], s_tm[1], kv_tile(sh, vst), j > 0);
+        if (more) {
+          issue_s(s_tm[1], q_tile(sh, 1), kv_tile(sh, kst));
+          mma_commit(smem_u32(sh.bars + kBarSFull + 1));
+        } else {
+          mma_commit(smem_u32(sh.bars + kBarOFull + 1));
+        }
+      }
+      mma_commit(smem_u32(sh.bars + kBarKVEmpty + vst));
+      if (more) mma_commit(smem_u32(sh.bars + kBarKVEmpty + kst));
+      if (j + 2 == n) mma_commit(smem_u32(sh.bars + kBarQEmpty));
+    }
+  }
+  // all issued MMAs complete before TMEM is released
+  mma_commit(smem_u32(sh.bars + kBarMmaDone));
+  const uint32_t addr = smem_u32(sh.bars + kBarMmaDone);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(addr, 0) && global_timer_ns() - t0 < p.timeout_ns) {
+  }
+}
+
+__device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, uint32_t tmem, int t, int u0, int u1) {
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int row_in_tile = (warp % 4) * 32 + lane;
+  const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
+  const uint32_t s_tm = tmem + lane_off + uint32_t(128 * t);
+  const uint32_t o_tm = tmem + lane_off + uint32_t(256 + 128 * t);
+  const float sl2 = p.scale_log2;
+  int s_cnt = 0, o_cnt = 0;
+  for (int u = u0; u < u1; ++u) {
+    const wf_plan_unit unit = p.units[u];
+    const int rows_here = p.C - unit.pair * 256 - 128 * t;
+    if (rows_here <= 0) continue;  // dead tile: the MMA thread skips it too
+    const wf_plan_chunk c = load_chunk(p.chunks + unit.chunk);
+    float m_ref = -INFINITY;  // reference max (log2 units)
+    float l = 0.f;
+    for (int j = 0; j < c.key_tiles; ++j) {
+      int32_t tok, valid;
+      key_tile(c, j, tok, valid);
+      if (!wait_bar(sh, p, kBarSFull + t, s_cnt & 1, 20 + t)) return;
+      ++s_cnt;
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(s_tm + 32 * q4, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s[32 * q4 + x] = __uint_as_float(r[x]);
+      }
+      tmem_wait_ld();
+      if (valid < 128) {
+#pragma unroll
+        for (int x = 0; x < 128; ++x)
+          if (x >= valid) s[x] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int x = 1; x < 128; ++x) mx = fmaxf(mx, s[x]);
+      const float m_new = fmaxf(m_ref, mx * sl2);
+      if (j == 0) {
+        m_ref = m_new;
+      } else {
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? fast_exp2(m_ref - m_new) : 1.0f;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t r[32];
+            tmem_ld32(o_tm + 32 * q4, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+            tmem_st32(o_tm + 32 * q4, r);
+          }
+          tmem_wait_st();
+          if (need) {
+            l *= alpha;
+            m_ref = m_new;
+          }
+        }
+      }
+      const float neg_m = -m_ref;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float p0 = fast_exp2(fmaf(s[32 * q4 + 2 * x], sl2, neg_m));
+          const float p1 = fast_exp2(fmaf(s[32 * q4 + 2 * x + 1], sl2, neg_m));
+          l += p0 + p1;
+          pk[x] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_tm + 16 * q4, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(sh.bars + kBarPFull + t));
+    }
+    // epilogue: O / l -> bf16 rows of this tile
+    if (!wait_bar(sh, p, kBarOFull + t, o_cnt & 1, 24 + t)) return;
+    ++o_cnt;
+    tc_fence_after();
+    const float inv_l = 1.0f / l;
+    const int32_t qtok = unit.chunk * p.C + unit.pair * 256 + 128 * t + row_in_tile;
+    const bool store = row_in_tile < rows_here;
+    uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t(qtok) * p.H + unit.head) * 128);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t r[32];
+      tmem_ld32(o_tm + 32 * q4, r);
+      tmem_wait_ld();
+      if (store) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv_l, __uint_as_float(r[8 * v + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_l, __uint_as_float(r[8 * v + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_l, __uint_as_float(r[8 * v + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_l, __uint_as_float(r[8 * v + 7]) * inv_l);
+          dst[4 * q4 + v] = w;
+        }
+      }
+    }
+    if (store && p.lse) p.lse[int64_t(unit.head) * p.rc + qtok] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+  }
+}
+
+__global__ void __maxnreg__(200)
+    attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Shared sh = carve_smem(smem_raw);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (warp == 9 && lane == 0) {
+    for (int b = 0; b < kNumBars; ++b) {
+      uint32_t count = 1;
+      if (b == kBarPFull || b == kBarPFull + 1) count = 128;
+      mbar_init(smem_u32(sh.bars + b), count);
+    }
+    *sh.abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(sh.tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sh.tmem_slot;
+  const int u0 = __ldg(p.cta_off + blockIdx.x);
+  const int u1 = __ldg(p.cta_off + blockIdx.x + 1);
+
+  if (warp < 8) {
+    softmax_role(sh, p, tmem, warp / 4, u0, u1);
+  } else if (warp == 8) {
+    if (lane == 0) mma_issuer(sh, p, tmem, u0, u1);
+    __syncwarp();
+  } else if (lane == 0) {
+    producer(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [tokens, H, 128] bf16 viewed as 3-D (dim, head, token); box = 64 dims x 1 head x 128 tokens.
+bool make_tmap(CUtensorMap* tm, const void* base, int64_t tokens, int32_t H) {
+  auto encode = get_encode();
+  if (!encode) return false;
+  cuuint64_t dims[3] = {128, cuuint64_t(H), cuuint64_t(tokens)};
+  cuuint64_t strides[2] = {128 * 2, cuuint64_t(H) * 128 * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Launch the tcgen05 path; arguments were validated by the caller.
+wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_rot, const void* k_pool,
+                            const void* v_pool, void* out, float* lse, float scale, void* workspace,
+                            uint64_t timeout_ns, cudaStream_t stream) {
+  static int attr_done[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WF_ERR_CUDA;
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(attn_fwd_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return WF_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q_rot, int64_t(h->R) * h->C, h->H) || !make_tmap(&tk, k_pool, int64_t(h->S) * h->C, h->H) ||
+      !make_tmap(&tv, v_pool, int64_t(h->S) * h->C, h->H))
+    return WF_ERR_CUDA;
+  Params p;
+  p.chunks = reinterpret_cast<const wf_plan_chunk*>(dev_plan + h->off_chunks);
+  p.units = reinterpret_cast<const wf_plan_unit*>(dev_plan + h->off_units);
+  p.cta_off = reinterpret_cast<const int32_t*>(dev_plan + h->off_cta);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = static_cast<wf_dev_status*>(workspace);
+  p.H = h->H;
+  p.C = h->C;
+  p.rc = h->R * h->C;
+  p.scale_log2 = float(double(scale) * 1.4426950408889634);
+  p.timeout_ns = timeout_ns;
+  attn_fwd_sm100<<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+}  // namespace wf

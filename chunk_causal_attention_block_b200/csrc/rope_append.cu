@@ -1,0 +1,180 @@
+// wf_rope3d_append: 3D rotary embedding of the round's new Q and K, fused
+// with the append of K'/V into the ring pool.
+//
+// HBM-bound: per (token, head) row it reads Q, K, V and writes Q', K', V
+// (6 * D * elem bytes).  Each thread moves one 16-byte vector of each tensor;
+// a warp covers consecutive vectors, so every load and store is a fully
+// coalesced 512-byte run.  The rotation runs in fp64 from the plan's fp64
+// cos/sin tables (L1-resident, a few KB) and is rounded once to the storage
+// type: fp64 -> fp32 with round-to-odd, then fp32 -> bf16 to nearest even,
+// which equals direct nearest-even rounding of the fp64 value (Boldo and
+// Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms
+// using rounding to odd", IEEE TC 2008: rounding to odd in a format with at
+// least two more bits makes the second rounding correct).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "wf.h"
+#include "wf_plan.h"
+
+namespace {
+
+struct RopeParams {
+  int32_t H, D, fh, fw, F, C, R, Pt, Ph, Pw;
+  int32_t slot[WF_MAX_INROUND];
+  const double2* tab_t;  // [R*F][Pt]
+  const double2* tab_h;  // [fh][Ph]
+  const double2* tab_w;  // [fw][Pw]
+  int64_t nvec;          // vectors in the new tensors
+};
+
+__device__ __forceinline__ float f64_to_f32_round_odd(double x) {
+  float r = __double2float_rz(x);
+  if (double(r) != x) r = __int_as_float(__float_as_int(r) | 1);
+  return r;
+}
+
+__device__ __forceinline__ void rotate_pair(double x, double y, double2 cs, double& xr, double& yr) {
+  // same operation order as a plain fp64 evaluation of x*c - y*s, x*s + y*c
+  xr = __dsub_rn(__dmul_rn(x, cs.x), __dmul_rn(y, cs.y));
+  yr = __dadd_rn(__dmul_rn(x, cs.y), __dmul_rn(y, cs.x));
+}
+
+template <typename T>
+struct Pack;
+
+template <>
+struct Pack<__nv_bfloat16> {
+  static constexpr int kElems = 8;
+  __device__ static void unpack(const uint4& v, double* out) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(p[i]);
+      out[2 * i] = f.x;
+      out[2 * i + 1] = f.y;
+    }
+  }
+  __device__ static uint4 pack(const double* in) {
+    uint4 v;
+    __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      p[i] = __floats2bfloat162_rn(f64_to_f32_round_odd(in[2 * i]), f64_to_f32_round_odd(in[2 * i + 1]));
+    return v;
+  }
+};
+
+template <>
+struct Pack<float> {
+  static constexpr int kElems = 4;
+  __device__ static void unpack(const uint4& v, double* out) {
+    const float* p = reinterpret_cast<const float*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out[i] = p[i];
+  }
+  __device__ static uint4 pack(const double* in) {
+    uint4 v;
+    float* p = reinterpret_cast<float*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = __double2float_rn(in[i]);
+    return v;
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) rope3d_append_kernel(RopeParams p, const uint4* __restrict__ q,
+                                                            const uint4* __restrict__ k,
+                                                            const uint4* __restrict__ v,
+                                                            uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
+                                                            uint4* __restrict__ v_pool) {
+  constexpr int E = Pack<T>::kElems;
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= p.nvec) return;
+  const uint4 qv = __ldcs(q + e);
+  const uint4 kv = __ldcs(k + e);
+  const uint4 vv = __ldcs(v + e);
+
+  const int32_t vpr = p.D / E;                  // vectors per (token, head) row
+  const int32_t row = int32_t(e / vpr);         // token * H + head
+  const int32_t vin = int32_t(e - int64_t(row) * vpr);
+  const int32_t token = row / p.H;
+  const int32_t head = row - token * p.H;
+  const int32_t i = token / p.C;                // in-round chunk
+  const int32_t j = token - i * p.C;            // token inside the chunk
+  const int32_t fhw = p.fh * p.fw;
+  const int32_t f = j / fhw;
+  const int32_t l = j - f * fhw;
+  const int32_t hh = l / p.fw;
+  const int32_t ww = l - hh * p.fw;
+
+  double qd[E], kd[E];
+  Pack<T>::unpack(qv, qd);
+  Pack<T>::unpack(kv, kd);
+#pragma unroll
+  for (int u = 0; u < E / 2; ++u) {
+    const int32_t m = vin * (E / 2) + u;  // pair index in [0, D/2)
+    double2 cs;
+    if (m < p.Pt) {
+      cs = __ldg(p.tab_t + int64_t(i * p.F + f) * p.Pt + m);
+    } else if (m < p.Pt + p.Ph) {
+      cs = __ldg(p.tab_h + int64_t(hh) * p.Ph + (m - p.Pt));
+    } else {
+      cs = __ldg(p.tab_w + int64_t(ww) * p.Pw + (m - p.Pt - p.Ph));
+    }
+    rotate_pair(qd[2 * u], qd[2 * u + 1], cs, qd[2 * u], qd[2 * u + 1]);
+    rotate_pair(kd[2 * u], kd[2 * u + 1], cs, kd[2 * u], kd[2 * u + 1]);
+  }
+  const int64_t dst = ((int64_t(p.slot[i]) * p.C + j) * p.H + head) * vpr + vin;
+  __stcs(q_rot + e, Pack<T>::pack(qd));
+  __stcs(k_pool + dst, Pack<T>::pack(kd));
+  __stcs(v_pool + dst, vv);
+}
+
+bool misaligned(const void* ptr) { return reinterpret_cast<uintptr_t>(ptr) % 16 != 0; }
+
+}  // namespace
+
+extern "C" wf_status wf_rope3d_append(const void* host_plan, const void* dev_plan, const void* q, const void* k,
+                                      const void* v, void* q_rot, void* k_pool, void* v_pool,
+                                      wf_stream_t stream) {
+  if (!host_plan || !dev_plan || !q || !k || !v || !q_rot || !k_pool || !v_pool) return WF_ERR_INVALID_ARG;
+  const wf_plan_hdr* h = static_cast<const wf_plan_hdr*>(host_plan);
+  if (h->magic != WF_PLAN_MAGIC || h->version != WF_PLAN_VERSION) return WF_ERR_PLAN;
+  if (misaligned(dev_plan) || misaligned(q) || misaligned(k) || misaligned(v) || misaligned(q_rot) ||
+      misaligned(k_pool) || misaligned(v_pool))
+    return WF_ERR_ALIGNMENT;
+  const int elem = h->dtype == WF_BF16 ? 2 : 4;
+  if ((h->D * elem) % 16 != 0) return WF_ERR_UNSUPPORTED;
+
+  RopeParams p{};
+  p.H = h->H; p.D = h->D; p.fh = h->fh; p.fw = h->fw; p.F = h->F; p.C = h->C; p.R = h->R;
+  p.Pt = h->Pt; p.Ph = h->Ph; p.Pw = h->Pw;
+  const wf_plan_chunk* ch = reinterpret_cast<const wf_plan_chunk*>(static_cast<const uint8_t*>(host_plan) + h->off_chunks);
+  for (int i = 0; i < h->R; ++i) p.slot[i] = ch[i].slot;
+  const uint8_t* dp = static_cast<const uint8_t*>(dev_plan);
+  p.tab_t = reinterpret_cast<const double2*>(dp + h->off_rope_t);
+  p.tab_h = reinterpret_cast<const double2*>(dp + h->off_rope_h);
+  p.tab_w = reinterpret_cast<const double2*>(dp + h->off_rope_w);
+  p.nvec = int64_t(h->R) * h->C * h->H * h->D * elem / 16;
+  if (p.nvec == 0) return WF_OK;
+
+  const int threads = 256;
+  const int64_t blocks = (p.nvec + threads - 1) / threads;
+  if (blocks > 0x7FFFFFFF) return WF_ERR_CAPACITY;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint4* q4 = static_cast<const uint4*>(q);
+  const uint4* k4 = static_cast<const uint4*>(k);
+  const uint4* v4 = static_cast<const uint4*>(v);
+  uint4* qr4 = static_cast<uint4*>(q_rot);
+  uint4* kp4 = static_cast<uint4*>(k_pool);
+  uint4* vp4 = static_cast<uint4*>(v_pool);
+  if (h->dtype == WF_BF16)
+    rope3d_append_kernel<__nv_bfloat16><<<unsigned(blocks), threads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
+  else
+    rope3d_append_kernel<float><<<unsigned(blocks), threads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
+  if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
+  return WF_OK;
+}

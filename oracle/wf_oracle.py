@@ -281,4 +281,4 @@ def wave_round(q_raw, k_raw, v_raw, k_cache_raw, v_cache_raw, *, n0, F, fh, fw,
     lse = np.zeros((len(rows), H))
     for h in range(H):
         out[:, h], lse[:, h] = attention(qf[:, h], keys[:, h], vals[:, h], mask, scale)
-    return dict(q_rot=q_rot, k_rot=k_rot, k_cache_rot=kc_rot, v=vr, O=out, LSE=lse, rows=rows)
+    return dict(q_rot=q_rot, k_rot=k_rot, k_cache_rot=kc_rot, v=vr, v_cache=vc, O=out, LSE=lse, rows=rows)
