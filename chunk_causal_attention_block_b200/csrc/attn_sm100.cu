@@ -37,6 +37,8 @@
 #include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 
 #include "sm100_ptx.cuh"
 #include "wf.h"
@@ -411,7 +413,10 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
   }
 }
 
-__global__ void __maxnreg__(200)
+#ifndef WF_ATTN_MAXNREG
+#define WF_ATTN_MAXNREG 168
+#endif
+__global__ void __maxnreg__(WF_ATTN_MAXNREG)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -461,14 +466,26 @@ __global__ void __maxnreg__(200)
 
 // ---------------------------------------------------------------- host
 
+// WF_VERBOSE=1 in the environment prints the failing CUDA step to stderr.
+bool report(const char* step, int err) {
+  static const int verbose = [] {
+    const char* v = std::getenv("WF_VERBOSE");
+    return v && v[0] == '1';
+  }();
+  if (verbose) std::fprintf(stderr, "[libwf] %s failed: error %d\n", step, err);
+  return false;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
+    const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess) {
+      report("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", int(e) * 1000 + int(q));
       return nullptr;
+    }
     fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   }
   return fn;
@@ -482,9 +499,10 @@ bool make_tmap(CUtensorMap* tm, const void* base, int64_t tokens, int32_t H) {
   cuuint64_t strides[2] = {128 * 2, cuuint64_t(H) * 128 * 2};
   cuuint32_t box[3] = {64, 1, 128};
   cuuint32_t estr[3] = {1, 1, 1};
-  return encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? true : report("cuTensorMapEncodeTiled", int(r));
 }
 
 }  // namespace
@@ -497,9 +515,12 @@ wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WF_ERR_CUDA;
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_fwd_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
+    const cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) {
+      report(cudaGetErrorString(e), int(e));
+      cudaGetLastError();
       return WF_ERR_CUDA;
+    }
     attr_done[dev] = 1;
   }
   CUtensorMap tq, tk, tv;
@@ -519,7 +540,19 @@ wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const
   p.scale_log2 = float(double(scale) * 1.4426950408889634);
   p.timeout_ns = timeout_ns;
   attn_fwd_sm100<<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    report(cudaGetErrorString(e), int(e));
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_sm100) == cudaSuccess) {
+      char msg[256];
+      std::snprintf(msg, sizeof(msg), "attributes: regs %d, max threads %d, static smem %zu, max dyn smem %d",
+                    fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.maxDynamicSharedSizeBytes);
+      report(msg, 0);
+    }
+    return WF_ERR_CUDA;
+  }
+  return WF_OK;
 }
 
 }  // namespace wf
