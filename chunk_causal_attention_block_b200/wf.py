@@ -28,7 +28,7 @@ WF_SYNTH_Q, WF_SYNTH_K, WF_SYNTH_V = 1, 2, 3
 # exported symbols, in the order include/wf.h and include/wf_synth.h declare them
 EXPORTS = ("wf_plan_bytes", "wf_plan_round", "wf_rope3d_append", "wf_attn_workspace_bytes",
            "wf_attn_workspace_init", "wf_attn_workspace_status", "wf_chunk_causal_attn",
-           "wf_status_string", "wf_version", "wf_synth_fill")
+           "wf_chunk_causal_attn_noalloc", "wf_status_string", "wf_version", "wf_synth_fill")
 
 
 class WfError(RuntimeError):
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.wf_attn_workspace_status.restype = i32
         L.wf_chunk_causal_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp]
         L.wf_chunk_causal_attn.restype = i32
+        L.wf_chunk_causal_attn_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp]
+        L.wf_chunk_causal_attn_noalloc.restype = i32
         L.wf_status_string.argtypes, L.wf_status_string.restype = [i32], ctypes.c_char_p
         L.wf_version.argtypes, L.wf_version.restype = [], i32
         L.wf_synth_fill.argtypes = [vp, i32, u64, i32, i64, i64, i32, i32, i32, i32, i32, vp]
@@ -164,6 +166,14 @@ def wf_chunk_causal_attn(host_plan, dev_plan, q_rot, k_pool, v_pool, out, lse=No
     _check(lib().wf_chunk_causal_attn(_ptr(host_plan), _ptr(dev_plan), _ptr(q_rot), _ptr(k_pool), _ptr(v_pool),
                                       _ptr(out), _ptr(lse), float(softmax_scale), _ptr(workspace), wb,
                                       _stream(stream)), "wf_chunk_causal_attn")
+
+
+def wf_chunk_causal_attn_noalloc(host_plan, dev_plan, q_rot, k_pool, v_pool, out, lse=None, softmax_scale=0.0,
+                                 stream=None):
+    """wf_chunk_causal_attn without a caller workspace (library-held static scratch)."""
+    _check(lib().wf_chunk_causal_attn_noalloc(_ptr(host_plan), _ptr(dev_plan), _ptr(q_rot), _ptr(k_pool),
+                                              _ptr(v_pool), _ptr(out), _ptr(lse), float(softmax_scale),
+                                              _stream(stream)), "wf_chunk_causal_attn_noalloc")
 
 
 def wf_synth_fill(dst, dtype, seed, tensor, tag, n_first, nchunks, C, H, D, kscale=False, stream=None):

@@ -26,7 +26,8 @@
  *   the plan's dtype (bf16 or fp32) for all of them.
  * - The caller owns every buffer.  The library never allocates or frees
  *   memory and keeps no state between calls except a per-device cache of
- *   kernel attributes.
+ *   kernel attributes (and the static scratch that
+ *   wf_chunk_causal_attn_noalloc documents).
  * - Device pointers must be 16-byte aligned; otherwise WF_ERR_ALIGNMENT.
  * - Every call is asynchronous on `stream` (NULL = legacy default stream) and
  *   never synchronises.  Argument errors are detected on the host before any
@@ -190,6 +191,36 @@ wf_status wf_chunk_causal_attn(const void* host_plan, const void* dev_plan,
                                const void* q_rot, const void* k_pool, const void* v_pool,
                                void* out, float* lse, float softmax_scale,
                                void* workspace, size_t workspace_bytes, wf_stream_t stream);
+
+/*
+ * wf_chunk_causal_attn_noalloc -- wf_chunk_causal_attn for callers that cannot
+ * allocate device memory.  The pages have no counterpart: this is an
+ * integration aid of this library, not part of the method.
+ *
+ * Some callers cannot call cudaMalloc: a serving engine or plugin host that
+ * reserves all of a GPU's memory for its own pool when it starts and forbids
+ * side allocations, or code that runs where allocating is not allowed.  This
+ * call takes the same inputs and outputs as wf_chunk_causal_attn but no
+ * workspace: the attention's scratch (its 256-byte status block) lives in a
+ * 4096-byte array in device memory that the library reserves on every GPU it
+ * is loaded on and keeps until the process exits.
+ *
+ * - The first call on a device looks up that array's device address (with the
+ *   device current) and caches it; make that first call before any stream
+ *   capture.  The call itself allocates nothing.
+ * - Each call zeroes the status block on `stream` before launching.  A wait
+ *   that times out is recorded there but is not returned by this call (it
+ *   returns once the kernel is queued); callers that need the device status
+ *   use wf_chunk_causal_attn with their own workspace.
+ * - Every call shares the one array: calls that overlap on the GPU (different
+ *   streams, not ordered) race on it.
+ * Errors: as wf_chunk_causal_attn, plus WF_ERR_CAPACITY if the plan's
+ * workspace need exceeds the 4096-byte array and WF_ERR_CUDA if the address
+ * look-up or the zeroing fails.
+ */
+wf_status wf_chunk_causal_attn_noalloc(const void* host_plan, const void* dev_plan,
+                                       const void* q_rot, const void* k_pool, const void* v_pool,
+                                       void* out, float* lse, float softmax_scale, wf_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* wf_status_string(wf_status status);
