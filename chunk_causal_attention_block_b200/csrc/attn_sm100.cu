@@ -8,11 +8,15 @@
 // loaded.  Only the last tile of a run can be ragged; its extra columns are
 // masked to -inf.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for query tile 0 (thread = one TMEM lane = one row)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    tcgen05.mma issue (lane 0) and TMEM allocation (whole warp)
-//   warp  9    TMA producer (lane 0)
+//   warp  9    TMA producer (lane 0); warps 10-11 idle
+// The block launches at 168 registers per thread (the most that three warps
+// per SM sub-partition allow); the control warpgroup then gives registers
+// back (setmaxnreg.dec to 56) and the softmax warpgroups take them
+// (setmaxnreg.inc to 224): 2*128*224 + 128*56 = 384*168.
 // TMEM (512 columns x 128 lanes x 32 bit):
 //   S_t = Q_t K^T at columns [128t, 128t+128), fp32; P_t (bf16 pairs) is
 //   written over the first 64 of them; O_t at [256+128t, 256+128t+128).
@@ -48,7 +52,13 @@ namespace wf {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr uint32_t kSoftmaxRegs = 224;
+constexpr uint32_t kControlRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * 168, "register split must match launch");
+// Pairs of score columns whose exp2 runs on the FMA pipe instead of MUFU:
+// bit k set = pair k of every 8 (3 of 8, i.e. 37.5% of the exponentials).
+constexpr uint32_t kPolyPairs = 0x25u;
 constexpr int kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr int kHalfBytes = kTileBytes / 2; // one 64-column (128-byte) half
 constexpr int kSmemBytes = 1024 + 2 * kTileBytes + kStages * kTileBytes + 256;
@@ -151,6 +161,29 @@ __device__ __forceinline__ wf_plan_chunk load_chunk(const wf_plan_chunk* p) {
   return c;
 }
 
+// 2^x for two values on the FMA pipe: x = j + f with j = rint(x) (the
+// 1.5*2^23 shift trick) and f in [-1/2, 1/2]; 2^f by a cubic fitted here to
+// 2^f on [-1/2, 1/2] (Lawson-reweighted least squares on relative error, max
+// relative error 7.5e-5 in fp32, far below the 2^-9 of the bf16 P it feeds);
+// 2^j is added to the exponent field.  x is clamped at -125 so the result
+// stays a normal number (2^-125 is 0 for all purposes here).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.24261054396629333f, c3 = 0.05517132207751274f;
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  // t's low mantissa bits hold j (two's complement); shifting by 23 drops the shift constant's bits
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ---------------------------------------------------------------- roles
 
 __device__ __forceinline__ void producer(const Shared& sh, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
@@ -209,28 +242,49 @@ __device__ __forceinline__ void producer(const Shared& sh, const Params& p, cons
   }
 }
 
-__device__ __forceinline__ void issue_s(uint32_t s_tmem, const uint8_t* q, const uint8_t* k) {
-  const uint32_t qa = smem_u32(q), ka = smem_u32(k);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    // K-major, 128-byte swizzle: 16-element K slices are 32 bytes apart
-    // inside a 64-element half; the second half starts 16 KB later.
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    mma_ss(s_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), kIdescQK,
-           kk > 0 ? 1u : 0u);
-  }
+// The descriptor's start-address field holds (address >> 4) in its low 14
+// bits; every offset below stays inside one tile, so adding (offset >> 4) to
+// a base descriptor moves its start address without touching other fields.
+// MMA issue is fully unrolled with every per-slice descriptor offset an
+// immediate: a single thread issues the MMAs, and per-MMA address arithmetic
+// in a loop made issue (about 100 cycles per MMA) slower than the tensor core
+// (64 cycles per 128x128x16 MMA).  Offsets are in 16-byte units and stay
+// inside one tile, so they never carry out of the start-address field.
+template <int kk>
+struct SliceOff {
+  // K-major, 128-byte swizzle: 16-element K slices are 32 bytes apart inside
+  // a 64-element half; the second half starts 16 KB later.
+  static constexpr uint32_t kKMajor = uint32_t(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+  // V is MN-major (head_dim contiguous): 16 keys = 2 KB further on; the two
+  // 64-column halves are 16 KB apart (leading byte offset), 8-key groups 1 KB
+  // apart (stride byte offset).
+  static constexpr uint32_t kMNMajor = uint32_t((kk * 2048) >> 4);
+};
+
+template <int kk>
+__device__ __forceinline__ void issue_s_slice(uint32_t s_tmem, uint64_t qd, uint64_t kd) {
+  mma_ss_off<SliceOff<kk>::kKMajor, SliceOff<kk>::kKMajor>(s_tmem, qd, kd, kIdescQK, kk > 0 ? 1u : 0u);
+  if constexpr (kk < 7) issue_s_slice<kk + 1>(s_tmem, qd, kd);
+}
+
+template <int kk>
+__device__ __forceinline__ void issue_pv_slice(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd, uint32_t acc0) {
+  // P_t holds 2 bf16 per TMEM column: 16 keys = 8 columns
+  mma_ts_off<kk * 8, SliceOff<kk>::kMNMajor>(o_tmem, p_tmem, vd, kIdescPV, kk > 0 ? 1u : acc0);
+  if constexpr (kk < 7) issue_pv_slice<kk + 1>(o_tmem, p_tmem, vd, acc0);
+}
+
+__device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile) { return smem_desc_sw128(smem_u32(tile), 16, 1024); }
+__device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile) {
+  return smem_desc_sw128(smem_u32(tile), kHalfBytes, 1024);
+}
+
+__device__ __forceinline__ void issue_s(uint32_t s_tmem, uint64_t qd, const uint8_t* k) {
+  issue_s_slice<0>(s_tmem, qd, kmajor_desc(k));
 }
 
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, const uint8_t* v, bool accumulate) {
-  const uint32_t va = smem_u32(v);
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    // V is MN-major (head_dim contiguous): 16 keys = 2 KB further on; the two
-    // 64-column halves are 16 KB apart (leading byte offset), 8-key groups
-    // 1 KB apart (stride byte offset).  P_t holds 2 bf16 per column.
-    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), kIdescPV,
-           (accumulate || kk > 0) ? 1u : 0u);
-  }
+  issue_pv_slice<0>(o_tmem, p_tmem, mnmajor_desc(v), accumulate ? 1u : 0u);
 }
 
 __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, uint32_t tmem, int u0, int u1) {
@@ -239,6 +293,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
   bool ok = true;
   const uint32_t s_tm[2] = {tmem + 0, tmem + 128};
   const uint32_t o_tm[2] = {tmem + 256, tmem + 384};
+  const uint64_t qd0 = kmajor_desc(q_tile(sh, 0)), qd1 = kmajor_desc(q_tile(sh, 1));
   for (int u = u0; u < u1 && ok; ++u) {
     const wf_plan_unit unit = p.units[u];
     const int n = __ldg(&p.chunks[unit.chunk].key_tiles);
@@ -250,10 +305,10 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
     if (!wait_bar(sh, p, kBarKVFull + kst, (kv_it / kStages) & 1, 11)) { ok = false; break; }
     ++kv_it;
     tc_fence_after();
-    issue_s(s_tm[0], q_tile(sh, 0), kv_tile(sh, kst));
+    issue_s(s_tm[0], qd0, kv_tile(sh, kst));
     mma_commit(smem_u32(sh.bars + kBarSFull + 0));
     if (live1) {
-      issue_s(s_tm[1], q_tile(sh, 1), kv_tile(sh, kst));
+      issue_s(s_tm[1], qd1, kv_tile(sh, kst));
       mma_commit(smem_u32(sh.bars + kBarSFull + 1));
     }
     mma_commit(smem_u32(sh.bars + kBarKVEmpty + kst));
@@ -274,7 +329,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
       tc_fence_after();
       issue_pv(o_tm[0], s_tm[0], kv_tile(sh, vst), j > 0);
       if (more) {
-        issue_s(s_tm[0], q_tile(sh, 0), kv_tile(sh, kst));
+        issue_s(s_tm[0], qd0, kv_tile(sh, kst));
         mma_commit(smem_u32(sh.bars + kBarSFull + 0));
       } else {
         mma_commit(smem_u32(sh.bars + kBarOFull + 0));
@@ -286,7 +341,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
         tc_fence_after();
         issue_pv(o_tm[1], s_tm[1], kv_tile(sh, vst), j > 0);
         if (more) {
-          issue_s(s_tm[1], q_tile(sh, 1), kv_tile(sh, kst));
+          issue_s(s_tm[1], qd1, kv_tile(sh, kst));
           mma_commit(smem_u32(sh.bars + kBarSFull + 1));
         } else {
           mma_commit(smem_u32(sh.bars + kBarOFull + 1));
@@ -341,9 +396,15 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
         for (int x = 0; x < 128; ++x)
           if (x >= valid) s[x] = -INFINITY;
       }
-      float mx = s[0];
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-      for (int x = 1; x < 128; ++x) mx = fmaxf(mx, s[x]);
+      for (int x = 4; x < 128; x += 8) {
+        mx0 = max3f(mx0, s[x], s[x + 1]);
+        mx1 = max3f(mx1, s[x + 2], s[x + 3]);
+        mx2 = max3f(mx2, s[x + 4], s[x + 5]);
+        mx3 = max3f(mx3, s[x + 6], s[x + 7]);
+      }
+      const float mx = fmaxf(max3f(mx0, mx1, mx2), mx3);
       const float m_new = fmaxf(m_ref, mx * sl2);
       if (j == 0) {
         m_ref = m_new;
@@ -367,19 +428,45 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
           }
         }
       }
-      const float neg_m = -m_ref;
+      const float2 sl2x2 = make_float2(sl2, sl2);
+      const float2 negm2 = make_float2(-m_ref, -m_ref);
+      float2 lsum = make_float2(0.f, 0.f);
+      if (valid == 128) {
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float p0 = fast_exp2(fmaf(s[32 * q4 + 2 * x], sl2, neg_m));
-          const float p1 = fast_exp2(fmaf(s[32 * q4 + 2 * x + 1], sl2, neg_m));
-          l += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
+          for (int x = 0; x < 16; ++x) {
+            const int pi = 16 * q4 + x;
+            const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
+            float2 pr;
+            if ((kPolyPairs >> (pi & 7)) & 1u) {
+              pr = exp2_poly2(v);
+            } else {
+              pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
+            }
+            lsum = __fadd2_rn(lsum, pr);
+            pk[x] = pack_bf16x2(pr.x, pr.y);
+          }
+          tmem_st16(s_tm + 16 * q4, pk);
         }
-        tmem_st16(s_tm + 16 * q4, pk);
+      } else {
+        // ragged tile: masked columns hold -inf and must give exactly 0 (MUFU path only)
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int pi = 16 * q4 + x;
+            const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
+            const float2 pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
+            lsum = __fadd2_rn(lsum, pr);
+            pk[x] = pack_bf16x2(pr.x, pr.y);
+          }
+          tmem_st16(s_tm + 16 * q4, pk);
+        }
       }
+      l += lsum.x + lsum.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(sh.bars + kBarPFull + t));
@@ -413,10 +500,7 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
   }
 }
 
-#ifndef WF_ATTN_MAXNREG
-#define WF_ATTN_MAXNREG 168
-#endif
-__global__ void __maxnreg__(WF_ATTN_MAXNREG)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -449,12 +533,16 @@ __global__ void __maxnreg__(WF_ATTN_MAXNREG)
   const int u1 = __ldg(p.cta_off + blockIdx.x + 1);
 
   if (warp < 8) {
+    regs_increase<kSoftmaxRegs>();
     softmax_role(sh, p, tmem, warp / 4, u0, u1);
-  } else if (warp == 8) {
-    if (lane == 0) mma_issuer(sh, p, tmem, u0, u1);
-    __syncwarp();
-  } else if (lane == 0) {
-    producer(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
+  } else {
+    regs_decrease<kControlRegs>();
+    if (warp == 8) {
+      if (lane == 0) mma_issuer(sh, p, tmem, u0, u1);
+      __syncwarp();
+    } else if (warp == 9 && lane == 0) {
+      producer(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
+    }
   }
   tc_fence_before();
   __syncthreads();
