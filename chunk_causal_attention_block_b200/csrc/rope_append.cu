@@ -2,9 +2,10 @@
 // with the append of K'/V into the ring pool.
 //
 // HBM-bound: per (token, head) row it reads Q, K, V and writes Q', K', V
-// (6 * D * elem bytes).  Each thread moves one 16-byte vector of each tensor;
-// a warp covers consecutive vectors, so every load and store is a fully
-// coalesced 512-byte run.  The rotation runs in fp64 from the plan's fp64
+// (6 * D * elem bytes).  Each thread moves two 16-byte vectors of each
+// tensor; a warp covers consecutive vectors, so every load and store is a
+// fully coalesced 512-byte run.  Index decoding uses exact multiply-shift
+// reciprocals instead of integer division.  The rotation runs in fp64 from the plan's fp64
 // cos/sin tables (L1-resident, a few KB) and is rounded once to the storage
 // type: fp64 -> fp32 with round-to-odd, then fp32 -> bf16 to nearest even,
 // which equals direct nearest-even rounding of the fp64 value (Boldo and
@@ -21,8 +22,31 @@
 
 namespace {
 
+// n / d for 0 <= n < 2^31 by a multiply and a shift: with k = 32 + ceil(log2 d)
+// and m = ceil(2^k / d), n*m / 2^k exceeds n/d by less than 1/(2d), which
+// cannot carry past the next integer, so the quotient is exact.
+struct FastDiv {
+  uint64_t m;
+  uint32_t k, d;
+};
+
+FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  FastDiv f;
+  f.k = 32 + l;
+  f.m = uint64_t((((unsigned __int128)1 << f.k) + d - 1) / d);
+  f.d = d;
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return uint32_t((uint64_t(n) * f.m) >> f.k);  // n < 2^31, m < 2^33: no overflow
+}
+
 struct RopeParams {
   int32_t H, D, fh, fw, F, C, R, Pt, Ph, Pw;
+  FastDiv div_vpr, div_H, div_C, div_fhw, div_fw;
   int32_t slot[WF_MAX_INROUND];
   const double2* tab_t;  // [R*F][Pt]
   const double2* tab_h;  // [fh][Ph]
@@ -84,38 +108,29 @@ struct Pack<float> {
   }
 };
 
+// Rotate and store one 16-byte vector of Q and K (and copy V) given its flat
+// index e in the [R*C, H, D] tensors.
 template <typename T>
-__global__ void __launch_bounds__(256) rope3d_append_kernel(RopeParams p, const uint4* __restrict__ q,
-                                                            const uint4* __restrict__ k,
-                                                            const uint4* __restrict__ v,
-                                                            uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
-                                                            uint4* __restrict__ v_pool) {
+__device__ __forceinline__ void rope_vector(const RopeParams& p, uint32_t e, const uint4& qv, const uint4& kv,
+                                            const uint4& vv, uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
+                                            uint4* __restrict__ v_pool) {
   constexpr int E = Pack<T>::kElems;
-  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= p.nvec) return;
-  const uint4 qv = __ldcs(q + e);
-  const uint4 kv = __ldcs(k + e);
-  const uint4 vv = __ldcs(v + e);
-
-  const int32_t vpr = p.D / E;                  // vectors per (token, head) row
-  const int32_t row = int32_t(e / vpr);         // token * H + head
-  const int32_t vin = int32_t(e - int64_t(row) * vpr);
-  const int32_t token = row / p.H;
-  const int32_t head = row - token * p.H;
-  const int32_t i = token / p.C;                // in-round chunk
-  const int32_t j = token - i * p.C;            // token inside the chunk
-  const int32_t fhw = p.fh * p.fw;
-  const int32_t f = j / fhw;
-  const int32_t l = j - f * fhw;
-  const int32_t hh = l / p.fw;
-  const int32_t ww = l - hh * p.fw;
-
+  const uint32_t row = fdiv(e, p.div_vpr);                   // token * H + head
+  const uint32_t vin = e - row * p.div_vpr.d;
+  const uint32_t token = fdiv(row, p.div_H);
+  const uint32_t head = row - token * uint32_t(p.H);
+  const uint32_t i = fdiv(token, p.div_C);                   // in-round chunk
+  const uint32_t j = token - i * uint32_t(p.C);              // token inside the chunk
+  const uint32_t f = fdiv(j, p.div_fhw);
+  const uint32_t l = j - f * p.div_fhw.d;
+  const uint32_t hh = fdiv(l, p.div_fw);
+  const uint32_t ww = l - hh * uint32_t(p.fw);
   double qd[E], kd[E];
   Pack<T>::unpack(qv, qd);
   Pack<T>::unpack(kv, kd);
 #pragma unroll
   for (int u = 0; u < E / 2; ++u) {
-    const int32_t m = vin * (E / 2) + u;  // pair index in [0, D/2)
+    const int32_t m = int32_t(vin) * (E / 2) + u;  // pair index in [0, D/2)
     double2 cs;
     if (m < p.Pt) {
       cs = __ldg(p.tab_t + int64_t(i * p.F + f) * p.Pt + m);
@@ -127,10 +142,33 @@ __global__ void __launch_bounds__(256) rope3d_append_kernel(RopeParams p, const 
     rotate_pair(qd[2 * u], qd[2 * u + 1], cs, qd[2 * u], qd[2 * u + 1]);
     rotate_pair(kd[2 * u], kd[2 * u + 1], cs, kd[2 * u], kd[2 * u + 1]);
   }
-  const int64_t dst = ((int64_t(p.slot[i]) * p.C + j) * p.H + head) * vpr + vin;
+  const int64_t dst = ((int64_t(p.slot[i]) * p.C + j) * p.H + head) * p.div_vpr.d + vin;
   __stcs(q_rot + e, Pack<T>::pack(qd));
   __stcs(k_pool + dst, Pack<T>::pack(kd));
   __stcs(v_pool + dst, vv);
+}
+
+// Each thread moves two vectors, blockDim apart (both halves of the block
+// stay coalesced); all six loads are issued before any arithmetic.
+template <typename T>
+__global__ void __launch_bounds__(256) rope3d_append_kernel(RopeParams p, const uint4* __restrict__ q,
+                                                            const uint4* __restrict__ k,
+                                                            const uint4* __restrict__ v,
+                                                            uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
+                                                            uint4* __restrict__ v_pool) {
+  const int64_t e0 = int64_t(blockIdx.x) * (2 * blockDim.x) + threadIdx.x;
+  const int64_t e1 = e0 + blockDim.x;
+  if (e0 >= p.nvec) return;
+  const bool two = e1 < p.nvec;
+  const uint4 q0 = __ldcs(q + e0), k0 = __ldcs(k + e0), v0 = __ldcs(v + e0);
+  uint4 q1 = make_uint4(0, 0, 0, 0), k1 = q1, v1 = q1;
+  if (two) {
+    q1 = __ldcs(q + e1);
+    k1 = __ldcs(k + e1);
+    v1 = __ldcs(v + e1);
+  }
+  rope_vector<T>(p, uint32_t(e0), q0, k0, v0, q_rot, k_pool, v_pool);
+  if (two) rope_vector<T>(p, uint32_t(e1), q1, k1, v1, q_rot, k_pool, v_pool);
 }
 
 bool misaligned(const void* ptr) { return reinterpret_cast<uintptr_t>(ptr) % 16 != 0; }
@@ -160,9 +198,15 @@ extern "C" wf_status wf_rope3d_append(const void* host_plan, const void* dev_pla
   p.tab_w = reinterpret_cast<const double2*>(dp + h->off_rope_w);
   p.nvec = int64_t(h->R) * h->C * h->H * h->D * elem / 16;
   if (p.nvec == 0) return WF_OK;
+  if (p.nvec >= (int64_t(1) << 31)) return WF_ERR_CAPACITY;  // the divisions assume indices < 2^31
+  p.div_vpr = make_fastdiv(uint32_t(h->D * elem / 16));
+  p.div_H = make_fastdiv(uint32_t(h->H));
+  p.div_C = make_fastdiv(uint32_t(h->C));
+  p.div_fhw = make_fastdiv(uint32_t(h->fh * h->fw));
+  p.div_fw = make_fastdiv(uint32_t(h->fw));
 
   const int threads = 256;
-  const int64_t blocks = (p.nvec + threads - 1) / threads;
+  const int64_t blocks = (p.nvec + 2 * threads - 1) / (2 * threads);
   if (blocks > 0x7FFFFFFF) return WF_ERR_CAPACITY;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint4* q4 = static_cast<const uint4*>(q);
