@@ -56,9 +56,6 @@ constexpr int kThreads = 384;
 constexpr uint32_t kSoftmaxRegs = 224;
 constexpr uint32_t kControlRegs = 56;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * 168, "register split must match launch");
-// Pairs of score columns whose exp2 runs on the FMA pipe instead of MUFU:
-// bit k set = pair k of every 8 (3 of 8, i.e. 37.5% of the exponentials).
-constexpr uint32_t kPolyPairs = 0x25u;
 constexpr int kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr int kHalfBytes = kTileBytes / 2; // one 64-column (128-byte) half
 constexpr int kSmemBytes = 1024 + 2 * kTileBytes + kStages * kTileBytes + 256;
@@ -159,29 +156,6 @@ __device__ __forceinline__ wf_plan_chunk load_chunk(const wf_plan_chunk* p) {
   c.seg_tiles[1] = __ldg(&p->seg_tiles[1]);
   c.key_tiles = __ldg(&p->key_tiles);
   return c;
-}
-
-// 2^x for two values on the FMA pipe: x = j + f with j = rint(x) (the
-// 1.5*2^23 shift trick) and f in [-1/2, 1/2]; 2^f by a cubic fitted here to
-// 2^f on [-1/2, 1/2] (Lawson-reweighted least squares on relative error, max
-// relative error 7.5e-5 in fp32, far below the 2^-9 of the bf16 P it feeds);
-// 2^j is added to the exponent field.  x is clamped at -125 so the result
-// stays a normal number (2^-125 is 0 for all purposes here).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.9999281167984009f, c1 = 0.6932609677314758f;
-  constexpr float c2 = 0.24261054396629333f, c3 = 0.05517132207751274f;
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
-  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));
-  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  p = __ffma2_rn(p, f, make_float2(c1, c1));
-  p = __ffma2_rn(p, f, make_float2(c0, c0));
-  // t's low mantissa bits hold j (two's complement); shifting by 23 drops the shift constant's bits
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // ---------------------------------------------------------------- roles
@@ -396,15 +370,15 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
         for (int x = 0; x < 128; ++x)
           if (x >= valid) s[x] = -INFINITY;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      float mxs[8];
 #pragma unroll
-      for (int x = 4; x < 128; x += 8) {
-        mx0 = max3f(mx0, s[x], s[x + 1]);
-        mx1 = max3f(mx1, s[x + 2], s[x + 3]);
-        mx2 = max3f(mx2, s[x + 4], s[x + 5]);
-        mx3 = max3f(mx3, s[x + 6], s[x + 7]);
+      for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(s[c], s[c + 8]);
+#pragma unroll
+      for (int x = 16; x < 128; x += 16) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
       }
-      const float mx = fmaxf(max3f(mx0, mx1, mx2), mx3);
+      const float mx = fmaxf(max3f(mxs[0], mxs[1], mxs[2]), max3f(mxs[3], max3f(mxs[4], mxs[5], mxs[6]), mxs[7]));
       const float m_new = fmaxf(m_ref, mx * sl2);
       if (j == 0) {
         m_ref = m_new;
@@ -428,45 +402,28 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
           }
         }
       }
+      // exp2 on MUFU for every score (an FMA-pipe polynomial for part of them
+      // measured slower here); four independent partial sums keep the row sum
+      // off one serial chain of adds.  Masked columns hold -inf: ex2 gives +0.
       const float2 sl2x2 = make_float2(sl2, sl2);
       const float2 negm2 = make_float2(-m_ref, -m_ref);
-      float2 lsum = make_float2(0.f, 0.f);
-      if (valid == 128) {
+      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const int pi = 16 * q4 + x;
-            const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
-            float2 pr;
-            if ((kPolyPairs >> (pi & 7)) & 1u) {
-              pr = exp2_poly2(v);
-            } else {
-              pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
-            }
-            lsum = __fadd2_rn(lsum, pr);
-            pk[x] = pack_bf16x2(pr.x, pr.y);
-          }
-          tmem_st16(s_tm + 16 * q4, pk);
+        for (int x = 0; x < 16; ++x) {
+          const int pi = 16 * q4 + x;
+          const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
+          const float2 pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
+          ls[x & 3] = __fadd2_rn(ls[x & 3], pr);
+          pk[x] = pack_bf16x2(pr.x, pr.y);
         }
-      } else {
-        // ragged tile: masked columns hold -inf and must give exactly 0 (MUFU path only)
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const int pi = 16 * q4 + x;
-            const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
-            const float2 pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
-            lsum = __fadd2_rn(lsum, pr);
-            pk[x] = pack_bf16x2(pr.x, pr.y);
-          }
-          tmem_st16(s_tm + 16 * q4, pk);
-        }
+        tmem_st16(s_tm + 16 * q4, pk);
       }
-      l += lsum.x + lsum.y;
+      const float2 l01 = __fadd2_rn(ls[0], ls[1]), l23 = __fadd2_rn(ls[2], ls[3]);
+      const float2 lt = __fadd2_rn(l01, l23);
+      l += lt.x + lt.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(sh.bars + kBarPFull + t));

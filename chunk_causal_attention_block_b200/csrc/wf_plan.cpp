@@ -199,7 +199,11 @@ extern "C" wf_status wf_plan_round(const wf_round_desc* desc, void* host_plan, s
         for (int p = 0; p < g.q_pairs; ++p) {
           const int32_t rows = std::min(WF_Q_PAIR, g.C - WF_Q_PAIR * p);
           const int32_t live = rows <= WF_Q_TILE ? 1 : 2;
-          units.push_back({i, hh, p, ch[i].key_tiles * live});
+          // A unit's time is set by its per-key-tile pipeline latency, which
+          // a second live query tile only lengthens by about a tenth (its
+          // softmax overlaps the first tile's MMAs): weight 11 for two live
+          // tiles, 10 for one.
+          units.push_back({i, hh, p, ch[i].key_tiles * (9 + live)});
         }
     std::sort(units.begin(), units.end(), [](const wf_plan_unit& a, const wf_plan_unit& b) {
       if (a.cost != b.cost) return a.cost > b.cost;
@@ -207,24 +211,76 @@ extern "C" wf_status wf_plan_round(const wf_round_desc* desc, void* host_plan, s
       if (a.head != b.head) return a.head < b.head;
       return a.pair < b.pair;
     });
+    // Greedy start: each unit, longest first, to the least-loaded bin
+    // (lowest index on ties).
     using Bin = std::pair<int64_t, int32_t>;  // (load, index): min-heap pops lowest load, then index
     std::priority_queue<Bin, std::vector<Bin>, std::greater<Bin>> heap;
     for (int32_t c = 0; c < g.G; ++c) heap.push({0, c});
-    std::vector<int32_t> owner(units.size());
-    std::vector<int32_t> count(g.G, 0);
+    std::vector<std::vector<wf_plan_unit>> bins(g.G);
+    std::vector<int64_t> load(g.G, 0);
     for (size_t u = 0; u < units.size(); ++u) {
       Bin b = heap.top();
       heap.pop();
-      owner[u] = b.second;
-      count[b.second]++;
-      heap.push({b.first + units[u].cost, b.second});
+      bins[b.second].push_back(units[u]);
+      load[b.second] += units[u].cost;
+      heap.push({load[b.second], b.second});
+    }
+    // Refinement: with ~6 large units per bin the greedy start leaves the
+    // heaviest bin ~10% above the mean.  Repeatedly move one unit out of the
+    // heaviest bin, or swap it for a lighter one, choosing the change that
+    // leaves the two bins' larger load smallest, from the lightest bin that
+    // offers any change lowering the maximum.  Deterministic: ties keep the
+    // first candidate in bin order, item order, move before swap.
+    for (int iter = 0; iter < 5000; ++iter) {
+      int32_t h = 0;
+      for (int32_t c = 1; c < g.G; ++c)
+        if (load[c] > load[h]) h = c;
+      std::vector<int32_t> order(g.G);
+      for (int32_t c = 0; c < g.G; ++c) order[c] = c;
+      std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return load[a] < load[b]; });
+      int64_t best = -1;
+      int32_t best_b = -1, best_x = -1, best_y = -1;
+      for (int32_t b : order) {
+        if (b == h) continue;
+        if (load[b] >= load[h]) break;
+        for (int32_t xi = 0; xi < int32_t(bins[h].size()); ++xi) {
+          const int64_t x = bins[h][xi].cost;
+          const int64_t mv = std::max(load[h] - x, load[b] + x);
+          if (mv < load[h] && (best < 0 || mv < best)) {
+            best = mv; best_b = b; best_x = xi; best_y = -1;
+          }
+          for (int32_t yi = 0; yi < int32_t(bins[b].size()); ++yi) {
+            const int64_t d = x - bins[b][yi].cost;
+            if (d <= 0) continue;
+            const int64_t sw = std::max(load[h] - d, load[b] + d);
+            if (sw < load[h] && (best < 0 || sw < best)) {
+              best = sw; best_b = b; best_x = xi; best_y = yi;
+            }
+          }
+        }
+        if (best >= 0) break;
+      }
+      if (best < 0) break;
+      const wf_plan_unit x = bins[h][best_x];
+      bins[h].erase(bins[h].begin() + best_x);
+      load[h] -= x.cost;
+      if (best_y >= 0) {
+        const wf_plan_unit y = bins[best_b][best_y];
+        bins[best_b].erase(bins[best_b].begin() + best_y);
+        load[best_b] -= y.cost;
+        bins[h].push_back(y);
+        load[h] += y.cost;
+      }
+      bins[best_b].push_back(x);
+      load[best_b] += x.cost;
     }
     int32_t* cta = reinterpret_cast<int32_t*>(base + g.off_cta);
-    cta[0] = 0;
-    for (int32_t c = 0; c < g.G; ++c) cta[c + 1] = cta[c] + count[c];
-    std::vector<int32_t> fill(cta, cta + g.G);
     wf_plan_unit* out = reinterpret_cast<wf_plan_unit*>(base + g.off_units);
-    for (size_t u = 0; u < units.size(); ++u) out[fill[owner[u]]++] = units[u];
+    cta[0] = 0;
+    for (int32_t c = 0; c < g.G; ++c) {
+      cta[c + 1] = cta[c] + int32_t(bins[c].size());
+      for (size_t k = 0; k < bins[c].size(); ++k) out[cta[c] + k] = bins[c][k];
+    }
   }
 
   if (dev_plan) {

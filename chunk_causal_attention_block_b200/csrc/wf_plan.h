@@ -30,7 +30,8 @@ struct wf_plan_chunk {
 static_assert(sizeof(wf_plan_chunk) == 56, "chunk record layout");
 
 // One attention work unit: query rows [pair*256, min(C, pair*256+256)) of
-// in-round chunk `chunk`, head `head`; cost = key_tiles * live 128-row tiles.
+// in-round chunk `chunk`, head `head`; cost = key_tiles * (9 + live 128-row
+// tiles): a unit's time is dominated by its per-key-tile pipeline latency.
 struct wf_plan_unit {
   int32_t chunk, head, pair, cost;
 };

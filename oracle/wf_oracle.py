@@ -179,7 +179,7 @@ def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas):
             for p in range(pairs):
                 rows = min(Q_PAIR, C - Q_PAIR * p)
                 live = 1 if rows <= Q_TILE else 2
-                units.append((i, h, p, chunks[i]["key_tiles"] * live))
+                units.append((i, h, p, chunks[i]["key_tiles"] * (9 + live)))
     units.sort(key=lambda u: (-u[3], -u[0], u[1], u[2]))
     loads = [0] * num_ctas
     per_cta = [[] for _ in range(num_ctas)]
@@ -187,6 +187,42 @@ def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas):
         c = min(range(num_ctas), key=lambda k: (loads[k], k))
         per_cta[c].append(u)
         loads[c] += u[3]
+    # refinement: move one unit out of the heaviest bin, or swap it for a
+    # lighter one, while that lowers the maximum; best change from the lightest
+    # bin offering any, ties to the first candidate (bin, item, move, swap)
+    for _ in range(5000):
+        h = max(range(num_ctas), key=lambda k: (loads[k], -k))
+        best = None
+        for b in sorted(range(num_ctas), key=lambda k: (loads[k], k)):
+            if b == h:
+                continue
+            if loads[b] >= loads[h]:
+                break
+            for xi, x in enumerate(per_cta[h]):
+                mv = max(loads[h] - x[3], loads[b] + x[3])
+                if mv < loads[h] and (best is None or mv < best[0]):
+                    best = (mv, b, xi, None)
+                for yi, y in enumerate(per_cta[b]):
+                    d = x[3] - y[3]
+                    if d <= 0:
+                        continue
+                    sw = max(loads[h] - d, loads[b] + d)
+                    if sw < loads[h] and (best is None or sw < best[0]):
+                        best = (sw, b, xi, yi)
+            if best is not None:
+                break
+        if best is None:
+            break
+        _, b, xi, yi = best
+        x = per_cta[h].pop(xi)
+        loads[h] -= x[3]
+        if yi is not None:
+            y = per_cta[b].pop(yi)
+            loads[b] -= y[3]
+            per_cta[h].append(y)
+            loads[h] += y[3]
+        per_cta[b].append(x)
+        loads[b] += x[3]
     return dict(C=C, wc_eff=wc_eff, first=first, chunks=chunks, units=units,
                 per_cta=per_cta, loads=loads, q_pairs=pairs)
 
