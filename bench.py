@@ -60,7 +60,7 @@ def load_peaks():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "wf_plan.h"):
+    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "wf_plan.h", "wf_plan.cpp"):
         with open(os.path.join(ROOT, "chunk_causal_attention_block_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
