@@ -80,6 +80,22 @@ def dram_traffic(config):
     return t.get("bytes_per_launch", {}).get(config)
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value over all ranks (the device time of the slowest replica)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(rank: int) -> int:
+    """Each replica draws its own inputs: seed 42 (the plugin's base_seed) + rank."""
+    return 42 + rank
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -212,7 +228,7 @@ def run_wf(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     W, K = args.warmup, args.steps
-    ro = Rollout(cfg, device=dev, want_lse=False, seed=42 + rank)
+    ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank))
     ro.prefill()
 
     # every step's inputs resident in HBM before timing (round r draws tag r)
@@ -265,11 +281,7 @@ def run_wf(args, rank, world, local_rank):
     code, detail = ro.device_status()
     if code != wf.WF_OK:
         raise RuntimeError(f"device status {wf.status_string(code)} {detail}")
-    ms_max = ms
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # End-to-end through the public calls with host buffers: every step copies
     # its Q/K/V from pinned host memory to the device and reads O back, inside
@@ -339,11 +351,7 @@ def run_wf(args, rank, world, local_rank):
         stream.wait_stream(down)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         elem = 2 if cfg.dtype == wf.WF_BF16 else 4
         plan_bytes = ro.host_plan.numel()
         e2e = {"value": cfg.attn_flops() * K * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
