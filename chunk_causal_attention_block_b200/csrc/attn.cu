@@ -111,15 +111,13 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const F32Params p) {
 
 bool misaligned(const void* ptr) { return reinterpret_cast<uintptr_t>(ptr) % 16 != 0; }
 
+// Limit of every bounded wait in the tensor-core kernel (WF_WAIT_TIMEOUT_MS,
+// default 2000 ms), read at each launch.
 uint64_t wait_timeout_ns() {
-  static uint64_t ns = 0;
-  if (!ns) {
-    const char* env = std::getenv("WF_WAIT_TIMEOUT_MS");
-    long ms = env ? std::atol(env) : 2000;
-    if (ms < 1) ms = 1;
-    ns = uint64_t(ms) * 1000000ull;
-  }
-  return ns;
+  const char* env = std::getenv("WF_WAIT_TIMEOUT_MS");
+  long ms = env ? std::atol(env) : 2000;
+  if (ms < 1) ms = 1;
+  return uint64_t(ms) * 1000000ull;
 }
 
 }  // namespace

@@ -76,6 +76,7 @@ struct Params {
   int32_t rc;            // R * C, the LSE row stride
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
+  int32_t stall_first_load;  // test hook: CTA 0 never issues its first K tile
 };
 
 // Barrier indices in the barrier block.
@@ -186,6 +187,12 @@ __device__ __forceinline__ void producer(const Shared& sh, const Params& p, cons
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int st = kv_it % kStages;
+        if (p.stall_first_load && blockIdx.x == 0 && kv_it == 0) {
+          // failure-detection test: this fill's barrier is never armed, so
+          // the MMA thread's bounded wait on it must expire
+          ++kv_it;
+          continue;
+        }
         if (!wait_bar(sh, p, kBarKVEmpty + st, ((kv_it / kStages) & 1) ^ 1, 2)) { ok = false; break; }
         const uint32_t bar = smem_u32(sh.bars + kBarKVFull + st);
         mbar_arrive_expect_tx(bar, kTileBytes);
@@ -584,6 +591,8 @@ wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const
   p.rc = h->R * h->C;
   p.scale_log2 = float(double(scale) * 1.4426950408889634);
   p.timeout_ns = timeout_ns;
+  const char* stall = std::getenv("WF_DEBUG_STALL_FIRST_LOAD");
+  p.stall_first_load = (stall && stall[0] == '1') ? 1 : 0;
   attn_fwd_sm100<<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

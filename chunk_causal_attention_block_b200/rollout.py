@@ -182,6 +182,33 @@ class Rollout:
     def device_status(self):
         return wf.wf_attn_workspace_status(self.workspace, self.stream)
 
+    # ------------------------------------------------------------- checkpoint / resume
+    def checkpoint(self) -> dict:
+        """Host copy of the stream state after the last completed round.
+
+        The ring pool is the only state carried between rounds: a round's plan
+        is a function of (n0, Wc, R, S) and its inputs are regenerated, so
+        resuming is restoring the pool and planning the next round.
+        """
+        self.stream.synchronize()
+        return {"round": self.round_index, "first_n0": self.first_n0, "seed": self.seed,
+                "k_pool": self.k_pool.cpu(), "v_pool": self.v_pool.cpu()}
+
+    def restore(self, state: dict):
+        """Load a checkpoint() taken from a rollout of the same configuration."""
+        for name in ("k_pool", "v_pool"):
+            src, dst = state[name], getattr(self, name)
+            if src.shape != dst.shape or src.dtype != dst.dtype:
+                raise ValueError(f"checkpoint {name} is {tuple(src.shape)} {src.dtype}, "
+                                 f"this rollout holds {tuple(dst.shape)} {dst.dtype}")
+        with torch.cuda.stream(self.stream):
+            self.k_pool.copy_(state["k_pool"], non_blocking=False)
+            self.v_pool.copy_(state["v_pool"], non_blocking=False)
+        self.first_n0 = int(state["first_n0"])
+        self.seed = int(state["seed"])
+        self.round_index = int(state["round"])
+        self.stream.synchronize()
+
 
 def default_scale(cfg: RoundConfig) -> float:
     return 1.0 / math.sqrt(cfg.D)
