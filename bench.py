@@ -373,6 +373,7 @@ def run_wf(args, rank, world, local_rank):
     peak = float(peaks["bf16_tflops"])
     traffic = dram_traffic(args.config)
     value = flops * K * world / (ms_max / 1e3) / 1e12
+    elem = 2 if cfg.dtype == wf.WF_BF16 else 4
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -383,7 +384,9 @@ def run_wf(args, rank, world, local_rank):
                    "inround_chunks": cfg.R, "queries_per_round": nq,
                    "visible_keys_per_chunk": cfg.visible_keys(), "global_batch": world,
                    "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (per-round Q/K/V 172 MB, K/V pool 316 MB, fresh inputs each step)"},
+                   "l2": (f"inputs larger than L2 (per-round Q/K/V {cfg.rope_bytes() / 2 / 1e6:.0f} MB, "
+                          f"K/V pool {2 * cfg.slots * cfg.C * cfg.H * cfg.D * elem / 1e6:.0f} MB, "
+                          "fresh inputs each step)")},
         "wave_rounds_per_s": K * world / (ms_max / 1e3),
         "attn_tflops_kernel": achieved,
         "pct_bf16_peak": {"of_spec_2250": 100 * achieved / 2250.0,

@@ -76,6 +76,21 @@ CONFIGS = {
                                 noise_t=(250, 500, 750, 1000), rounds=200, check_rounds=(0, 1, 21, 199)),
 }
 
+# Cache-refresh schedules: the round also carries the graduating chunk once
+# more at t=0 (the oldest in-round member), so the clean K/V it leaves in its
+# ring slot are those of the clean latent.  4-step schedule + refresh (R=5)
+# and 5-step schedule + refresh (R=6, steps evenly spaced: the pages print no
+# 5-step list).
+REFRESH_CONFIGS = {
+    "wan13b_refresh": RoundConfig("Wan2.1-1.3B-shaped 4-step round with cache refresh", H=12, D=128, fh=30, fw=52,
+                                  F=3, Wc=7, R=5, noise_t=(0, 250, 500, 750, 1000), rounds=16,
+                                  check_rounds=(0, 1, 15)),
+    "wan13b_5step_refresh": RoundConfig("Wan2.1-1.3B-shaped 5-step round with cache refresh", H=12, D=128, fh=30,
+                                        fw=52, F=3, Wc=7, R=6, noise_t=(0, 200, 400, 600, 800, 1000), rounds=16,
+                                        check_rounds=(0, 1, 15)),
+}
+CONFIGS.update(REFRESH_CONFIGS)
+
 
 class Rollout:
     """Device state of one stream: the K/V ring pool, the round's buffers, plan and workspace."""

@@ -145,6 +145,21 @@ def test_720p_200_round_rollout_sampled():
         ro, r, [17], rows, f"720p r{r}"))
 
 
+@pytest.mark.parametrize("name,heads", [("wan13b_refresh", [2, 9]), ("wan13b_5step_refresh", [4])])
+def test_cache_refresh_rounds_sampled(name, heads):
+    """Rounds whose oldest member is the graduating chunk re-run at t=0."""
+    cfg = CONFIGS[name]
+    rows = gc.sample_rows(cfg, extra=12)
+    rope = {}
+
+    def on_round(ro, r):
+        gc.check_attention(ro, r, heads, rows, f"{name} r{r}")
+        rope[r] = gc.check_rope_append(ro, r, heads[:1])
+
+    gc.run_rollout(cfg, cfg.check_rounds, on_round=on_round)
+    assert all(all(v == 0 for v in m.values()) for m in rope.values()), rope
+
+
 # ------------------------------------------------------------------ invariants and controls
 
 def test_later_chunks_never_touch_earlier_outputs():
