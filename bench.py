@@ -287,7 +287,10 @@ def run_wf(args, rank, world, local_rank):
     # its Q/K/V from pinned host memory to the device and reads O back, inside
     # the timed region.  Copies run on their own streams, double-buffered, so
     # the upload of step r+1 and the read-back of step r-1 overlap step r's
-    # kernels; events order every buffer reuse.
+    # kernels; events order every buffer reuse.  Each round's plan is built
+    # and copied on the upload stream with its inputs (two host and two
+    # device plan buffers): a plan copy queued on the compute stream would
+    # wait behind the 57 MB input uploads on the same copy engine.
     e2e = None
     if not args.no_e2e:
         nsets = min(4, W + K)
@@ -295,18 +298,23 @@ def run_wf(args, rank, world, local_rank):
         host_out = [torch.empty(nq, cfg.H, cfg.D, dtype=tdt).pin_memory() for _ in range(2)]
         dev_in = [tuple(torch.empty_like(inputs[0][0]) for _ in range(3)) for _ in range(2)]
         dev_out = [torch.empty(nq, cfg.H, cfg.D, dtype=tdt, device=dev) for _ in range(2)]
+        plan_bytes = max(wf.wf_plan_bytes(ro.desc(ro.n0_of(r))) for r in range(2 * (W + K) + 1))
+        host_plan = [torch.empty(plan_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        dev_plan = [torch.empty(plan_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
         del inputs
         torch.cuda.empty_cache()
         up = torch.cuda.Stream(dev)
         down = torch.cuda.Stream(dev)
-        in_free = [torch.cuda.Event() for _ in range(2)]     # RoPE/append done reading a set
-        in_ready = [torch.cuda.Event() for _ in range(2)]    # upload of a set done
+        in_free = [torch.cuda.Event() for _ in range(2)]     # attention done with a set (inputs, plan)
+        in_ready = [torch.cuda.Event() for _ in range(2)]    # upload of a set (plan + inputs) done
         out_ready = [torch.cuda.Event() for _ in range(2)]   # attention wrote an output buffer
         out_free = [torch.cuda.Event() for _ in range(2)]    # read-back of an output buffer done
 
         def upload(r):
             b = r % 2
+            in_ready[b].synchronize()  # the host plan buffer's previous copy has left
             up.wait_event(in_free[b])
+            wf.wf_plan_round(ro.desc(ro.n0_of(r)), host_plan[b], dev_plan[b], up)
             with torch.cuda.stream(up):
                 for dst, src in zip(dev_in[b], host_in[r % nsets]):
                     dst.copy_(src, non_blocking=True)
@@ -316,12 +324,12 @@ def run_wf(args, rank, world, local_rank):
             b = r % 2
             stream.wait_event(in_ready[b])
             ro.q, ro.k, ro.v = dev_in[b]
-            ro.plan_round(r)
+            ro.host_plan, ro.dev_plan = host_plan[b], dev_plan[b]
             ro.append()
-            in_free[b].record(stream)
             stream.wait_event(out_free[b])
             ro.out = dev_out[b]
             ro.attend()
+            in_free[b].record(stream)
             out_ready[b].record(stream)
 
         def download(r):
@@ -353,12 +361,11 @@ def run_wf(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         elem = 2 if cfg.dtype == wf.WF_BF16 else 4
-        plan_bytes = ro.host_plan.numel()
         e2e = {"value": cfg.attn_flops() * K * world / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": 3 * nq * cfg.H * cfg.D * elem + plan_bytes,
+               "h2d_bytes_per_step": 3 * nq * cfg.H * cfg.D * elem + wf.wf_plan_bytes(ro.desc(ro.n0_of(base + W))),
                "d2h_bytes_per_step": nq * cfg.H * cfg.D * elem,
                "ms_per_step": e_ms / K,
-               "overlap": "uploads of step r+1 and read-back of step r-1 overlap step r on two copy streams"}
+               "overlap": "plan + uploads of step r+1 and read-back of step r-1 overlap step r on two copy streams"}
         code, detail = ro.device_status()
         if code != wf.WF_OK:
             raise RuntimeError(f"device status {wf.status_string(code)} {detail}")
