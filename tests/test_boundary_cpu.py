@@ -138,6 +138,9 @@ PLAN_CASES = [
          num_ctas=148),
     dict(H=3, D=128, fh=5, fw=7, F=2, Wc=5, R=4, S=13, n0=2, noise_t=[0, 0, 500, 500], num_ctas=7),  # start
     dict(H=1, D=128, fh=1, fw=1, F=1, Wc=0, R=5, S=5, n0=11, noise_t=[0, 1, 2, 3, 4], num_ctas=2),   # C=1
+    # the most in-round chunks (16), ring wrapped
+    dict(H=1, D=128, fh=6, fw=7, F=1, Wc=3, R=16, S=19, n0=3 + 40, noise_t=[60 * i for i in range(16)],
+         num_ctas=148),
     # cache-refresh rounds: the oldest member at t=0 (4-step + refresh, 5-step + refresh), ring wrapped
     dict(H=12, D=128, fh=30, fw=52, F=3, Wc=7, R=5, S=12, n0=7 + 13, noise_t=[0, 250, 500, 750, 1000],
          num_ctas=148),

@@ -90,6 +90,8 @@ SMALL_BF16 = [
     RoundConfig("aligned", H=1, D=128, fh=16, fw=16, F=1, Wc=2, R=2, noise_t=(500, 1000)),
     # one token per chunk
     RoundConfig("C=1", H=2, D=128, fh=1, fw=1, F=1, Wc=5, R=4, noise_t=(250, 500, 750, 1000)),
+    # the most in-round chunks a round may hold (16), ragged 42-token chunks
+    RoundConfig("R=16", H=1, D=128, fh=6, fw=7, F=1, Wc=3, R=16, noise_t=tuple(60 * i for i in range(16))),
 ]
 
 
