@@ -284,17 +284,81 @@ def attention_bruteforce(q, k, v, mask, scale: float):
 
 
 # --------------------------------------------------------------------------
+# 8-bit scores: e4m3 codes with per-block scales
+# --------------------------------------------------------------------------
+# The 8-bit variant of the attention (the B200 counterpart of the 8-bit
+# attention backends the Wave Forcing abstract benchmarks against) quantizes
+# the rotated Q and K, not V: per (chunk, block of FP8_BLOCK consecutive
+# chunk-relative tokens, head) one fp32 scale = amax / 448, and every element
+# becomes the e4m3 value nearest x / scale.  Scores are products of the
+# dequantized values; P and V stay as in the 16-bit path.
+
+E4M3_MAX = 448.0   # largest finite e4m3 value (1.75 * 2^8)
+FP8_BLOCK = 128    # tokens per scale block
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Nearest-even rounding to OCP FP8 E4M3 (sign, 4 exponent bits with bias
+    7, 3 mantissa bits; normals from 2^-6, subnormals in steps of 2^-9; no
+    infinities), saturating to +-448 as a satfinite conversion does."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, e = np.frexp(a)                       # a = m * 2^e, m in [0.5, 1)
+    binade = np.maximum(e - 1, -6)           # subnormals share the 2^-6 binade's step
+    step = np.ldexp(1.0, binade - 3)         # 3 mantissa bits
+    r = np.minimum(np.rint(a / step) * step, E4M3_MAX)
+    return np.copysign(r, x)
+
+
+def fp8_block_quantize(x, C: int):
+    """x: [n*C, H, D] values (exact in fp32), n whole chunks of C tokens.
+
+    Per chunk, block b of tokens [b*FP8_BLOCK, min(C, (b+1)*FP8_BLOCK)) and
+    head: scale = fp32(amax / 448) (1 for an all-zero block), codes =
+    round_e4m3(fp32(x / scale)).  Both divisions are single fp32 divisions
+    rounded to nearest.  Returns (codes [n*C, H, D] as values, scales
+    [n, nblk, H] float64 holding fp32 values).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    T, H, D = x.shape
+    n = T // C
+    nblk = -(-C // FP8_BLOCK)
+    codes = np.zeros_like(x)
+    scales = np.zeros((n, nblk, H))
+    for c in range(n):
+        for b in range(nblk):
+            lo, hi = c * C + b * FP8_BLOCK, c * C + min(C, (b + 1) * FP8_BLOCK)
+            blk = x[lo:hi].astype(np.float32)                       # [tokens, H, D], exact
+            amax = np.abs(blk).max(axis=(0, 2))                      # [H]
+            sc = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+            scales[c, b] = sc
+            codes[lo:hi] = round_e4m3((blk / sc[None, :, None]).astype(np.float32))
+    return codes, scales
+
+
+def fp8_dequantize(codes, scales, C: int) -> np.ndarray:
+    """codes [n*C, H, D] times the scale of each element's block (exact in fp64)."""
+    T, H, D = codes.shape
+    tok = np.arange(T)
+    sc = scales[tok // C, (tok % C) // FP8_BLOCK]                    # [T, H]
+    return codes * sc[:, :, None]
+
+
+# --------------------------------------------------------------------------
 # one wave round
 # --------------------------------------------------------------------------
 
 def wave_round(q_raw, k_raw, v_raw, k_cache_raw, v_cache_raw, *, n0, F, fh, fw,
-               pairs, theta, dtype, scale=None, rows=None):
+               pairs, theta, dtype, scale=None, rows=None, fp8=False):
     """One wave round for the heads present in the inputs.
 
     q_raw/k_raw/v_raw: [R, C, H, D] raw in-round tensors (chunk i is global n0+i);
     k_cache_raw/v_cache_raw: [Wc_eff, C, H, D] raw K/V of cache chunks
     n0-Wc_eff .. n0-1 as they were when last appended.
     rows: optional in-round query indices (flat over R*C) to evaluate.
+    fp8: scores from block-quantized e4m3 Q and K (see fp8_block_quantize);
+    the codes and scales are returned as q8, q_scales, k8 (cache chunks then
+    in-round chunks) and k_scales.
     Returns dict with q_rot [R,C,H,D], k_rot [R,C,H,D], k_cache_rot, O [nrows,H,D],
     LSE [nrows,H] -- rotated tensors rounded to ``dtype``.
     """
@@ -312,9 +376,17 @@ def wave_round(q_raw, k_raw, v_raw, k_cache_raw, v_cache_raw, *, n0, F, fh, fw,
     vals = np.concatenate([vc, vr]).reshape(-1, H, D)
     rows = np.arange(R * C) if rows is None else np.asarray(rows)
     mask = visibility_mask(C, wc_eff, R, q_chunks=rows // C)
-    qf = q_rot.reshape(-1, H, D)[rows]
+    extra = {}
+    qall = q_rot.reshape(-1, H, D)
+    if fp8:
+        q8, qs = fp8_block_quantize(qall, C)
+        k8, ks = fp8_block_quantize(keys, C)
+        qall, keys = fp8_dequantize(q8, qs, C), fp8_dequantize(k8, ks, C)
+        extra = dict(q8=q8, q_scales=qs, k8=k8, k_scales=ks)
+    qf = qall[rows]
     out = np.zeros((len(rows), H, D))
     lse = np.zeros((len(rows), H))
     for h in range(H):
         out[:, h], lse[:, h] = attention(qf[:, h], keys[:, h], vals[:, h], mask, scale)
-    return dict(q_rot=q_rot, k_rot=k_rot, k_cache_rot=kc_rot, v=vr, v_cache=vc, O=out, LSE=lse, rows=rows)
+    return dict(q_rot=q_rot, k_rot=k_rot, k_cache_rot=kc_rot, v=vr, v_cache=vc, O=out, LSE=lse, rows=rows,
+                **extra)

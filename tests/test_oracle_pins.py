@@ -360,3 +360,94 @@ def test_wave_round_against_per_query_bruteforce():
                                                   1 / math.sqrt(D))
                 np.testing.assert_allclose(out["O"][i * C + j, h], ob[0], rtol=1e-12, atol=1e-13)
                 np.testing.assert_allclose(out["LSE"][i * C + j, h], lb[0], rtol=1e-12)
+
+
+# ------------------------------------------------------------------ 8-bit scores
+
+def _e4m3_decode(code: int):
+    """Value of an E4M3 code from the format's definition (None for NaN)."""
+    s, e, m = code >> 7, (code >> 3) & 15, code & 7
+    if e == 15 and m == 7:
+        return None
+    v = Fraction(m, 8) * Fraction(1, 64) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+    return -v if s else v
+
+
+def test_e4m3_codes_are_fixed_points_and_midpoints_go_to_even():
+    pos = sorted({_e4m3_decode(c) for c in range(128) if _e4m3_decode(c) is not None})
+    assert pos[0] == 0 and pos[1] == Fraction(1, 512) and pos[-1] == 448 and len(pos) == 127
+    vals = np.array([float(v) for v in pos])
+    assert np.array_equal(orc.round_e4m3(vals), vals)
+    assert np.array_equal(orc.round_e4m3(-vals), -vals)
+    even = {float(_e4m3_decode(c)): (c & 1) == 0 for c in range(127)}
+    for lo, hi in zip(pos[:-1], pos[1:]):
+        mid = (lo + hi) / 2
+        want = float(lo) if even[float(lo)] else float(hi)
+        assert orc.round_e4m3(float(mid)) == want, (lo, hi)
+        eps = (hi - lo) / 1024
+        assert orc.round_e4m3(float(mid - eps)) == float(lo)
+        assert orc.round_e4m3(float(mid + eps)) == float(hi)
+    # beyond the largest finite value the conversion saturates
+    assert np.array_equal(orc.round_e4m3([448.5, 464.0, 480.0, 1e9, -1e9]), [448, 448, 448, 448, -448])
+
+
+def test_e4m3_rounding_matches_torch_float8():
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(200_000) * np.exp2(rng.integers(-14, 9, 200_000))).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    t = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(orc.round_e4m3(x.astype(np.float64)), t)
+
+
+def test_fp8_block_quantize_hand_case():
+    # C = 130 tokens: block 0 = tokens 0..127, block 1 = tokens 128..129 (ragged); 2 heads, D = 4
+    C, H, D = 130, 2, 4
+    x = np.zeros((C, H, D))
+    x[5, 0] = [3.5, -1.0, 0.25, 0.0]          # head 0, block 0: amax 3.5 -> scale 2^-7 exactly
+    x[70, 0] = [-2.0, 1.5, 0.0, 0.125]
+    x[129, 0] = [0.75, 0.0, 0.0, -0.375]      # head 0, block 1: amax 0.75 -> scale fp32(0.75/448)
+    codes, scales = orc.fp8_block_quantize(x, C)
+    assert scales.shape == (1, 2, 2)
+    assert scales[0, 0, 0] == 2.0 ** -7
+    assert scales[0, 0, 1] == 1.0 and scales[0, 1, 1] == 1.0         # all-zero blocks
+    assert scales[0, 1, 0] == float(np.float32(0.75) / np.float32(448.0))
+    assert np.array_equal(codes[5, 0], [448.0, -128.0, 32.0, 0.0])   # x * 128, all representable
+    assert np.array_equal(codes[70, 0], [-256.0, 192.0, 0.0, 16.0])
+    assert abs(codes[129, 0, 0]) == 448.0                             # the block max maps to the largest code
+    assert codes[129, 0, 3] == orc.round_e4m3(np.float32(-0.375) / np.float32(scales[0, 1, 0]))
+    assert not codes[:, 1].any()
+    deq = orc.fp8_dequantize(codes, scales, C)
+    assert np.array_equal(deq[5, 0], x[5, 0]) and np.array_equal(deq[70, 0], x[70, 0])
+
+
+def test_fp8_dequantized_error_within_half_an_e4m3_step():
+    rng = np.random.default_rng(3)
+    C = 300
+    x = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(rng.standard_normal((2 * C, 3, 16)).astype(np.float32))) \
+        .astype(np.float64)
+    codes, scales = orc.fp8_block_quantize(x, C)
+    deq = orc.fp8_dequantize(codes, scales, C)
+    tok = np.arange(2 * C)
+    sc = scales[tok // C, (tok % C) // orc.FP8_BLOCK][:, :, None]
+    # half a step of the binade (relative 2^-4) for normals, 2^-10 * scale in the subnormal range,
+    # plus the fp32 rounding of x / scale (relative 2^-24)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, sc * 2.0 ** -10) * (1 + 2.0 ** -20)
+    assert (np.abs(deq - x) <= bound).all()
+
+
+def test_fp8_round_equals_16_bit_round_when_quantization_is_exact():
+    # inputs whose rotated values are e4m3-exact after scaling: a zero angle (n = 0, one token
+    # per chunk at position 0) and values that are small multiples of powers of two
+    rng = np.random.default_rng(11)
+    R, C, H, D = 1, 1, 2, 16
+    q = rng.integers(-7, 8, (R, C, H, D)) / 8.0
+    k = rng.integers(-7, 8, (R, C, H, D)) / 8.0
+    v = rng.standard_normal((R, C, H, D))
+    q[0, 0, :, 0] = 1.75
+    k[0, 0, :, 0] = 1.75                   # amax 1.75 -> scale 1.75/448 = 2^-8
+    kw = dict(n0=0, F=1, fh=1, fw=1, pairs=orc.rope_split(D), theta=10000.0, dtype="f32")
+    empty = np.zeros((0, C, H, D))
+    a = orc.wave_round(q, k, v, empty, empty, **kw)
+    b = orc.wave_round(q, k, v, empty, empty, fp8=True, **kw)
+    assert np.array_equal(b["q8"] * 2.0 ** -8, a["q_rot"].reshape(-1, H, D))
+    assert np.array_equal(a["O"], b["O"]) and np.array_equal(a["LSE"], b["LSE"])
