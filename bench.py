@@ -42,6 +42,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("wf", "reference"), default="wf")
     ap.add_argument("--config", default="wan13b_round")
+    ap.add_argument("--scores", choices=("bf16", "fp8"), default="bf16",
+                    help="fp8: e4m3 Q/K codes with block scales (quantization timed with RoPE/append)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -228,7 +230,7 @@ def run_wf(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     W, K = args.warmup, args.steps
-    ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank))
+    ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank), fp8=args.scores == "fp8")
     ro.prefill()
 
     # every step's inputs resident in HBM before timing (round r draws tag r)
@@ -384,7 +386,8 @@ def run_wf(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if cfg.dtype == wf.WF_BF16 else "f32",
+        "dtype": ("e4m3 scores, bf16 P/V/O" if args.scores == "fp8" else "bf16") if cfg.dtype == wf.WF_BF16
+        else "f32",
         "data": "synthetic (seeded Irwin-Hall(12) N(0,1) draws, seed 42 + rank, drawn on device before timing)",
         "config": {"workload": cfg.name, "heads": cfg.H, "head_dim": cfg.D,
                    "tokens_per_frame": cfg.fh * cfg.fw, "chunk_tokens": cfg.C, "cache_chunks": cfg.Wc,

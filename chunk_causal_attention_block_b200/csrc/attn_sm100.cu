@@ -64,6 +64,9 @@ constexpr float kRescaleThreshold = 8.0f;
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);
+// 8-bit scores: Q and K tiles of 128 tokens x 128 e4m3 codes (one 128-byte row each)
+constexpr uint32_t kIdescQK8 = idesc_e4m3_f32(128, 128);
+constexpr int kTile8Bytes = 128 * 128;
 
 struct Params {
   const wf_plan_chunk* chunks;
@@ -77,6 +80,10 @@ struct Params {
   float scale_log2;      // softmax scale * log2(e)
   uint64_t timeout_ns;
   int32_t stall_first_load;  // test hook: CTA 0 never issues its first K tile
+  // 8-bit scores only
+  const float* q_scales;     // [R, nblk, H]
+  const float* k_scales;     // [S, nblk, H]
+  int32_t S, nblk;           // pool slots; scale blocks (= key tiles) per chunk
 };
 
 // Barrier indices in the barrier block.
@@ -147,6 +154,35 @@ __device__ __forceinline__ void key_tile(const wf_plan_chunk& c, int j, int32_t&
   valid = left < 128 ? left : 128;
 }
 
+// 8-bit path: the key tiles are the chunks' scale blocks.  Tile j of a unit
+// whose oldest visible chunk sits in slot first_slot is block `blk` of
+// visible chunk j / nblk.
+__device__ __forceinline__ void key_tile_fp8(const Params& p, int first_slot, int j, int32_t& tok, int32_t& valid,
+                                             int32_t& slot, int32_t& blk) {
+  const int v = j / p.nblk;
+  blk = j - v * p.nblk;
+  slot = first_slot + v;  // v < nvis <= S
+  if (slot >= p.S) slot -= p.S;
+  tok = slot * p.C + blk * 128;
+  const int32_t left = p.C - blk * 128;
+  valid = left < 128 ? left : 128;
+}
+
+// Visible chunks are the consecutive global indices n - nvis + 1 .. n.
+__device__ __forceinline__ int first_visible_slot(const Params& p, const wf_plan_chunk* rec) {
+  const int64_t n = __ldg(&rec->n);
+  const int32_t nvis = __ldg(&rec->nvis);
+  return int((n - nvis + 1) % p.S);
+}
+
+template <bool kFp8>
+__device__ __forceinline__ int unit_key_tiles(const Params& p, const wf_plan_chunk* rec) {
+  if constexpr (kFp8)
+    return __ldg(&rec->nvis) * p.nblk;
+  else
+    return __ldg(&rec->key_tiles);
+}
+
 __device__ __forceinline__ wf_plan_chunk load_chunk(const wf_plan_chunk* p) {
   wf_plan_chunk c;
   c.seg_start[0] = __ldg(&p->seg_start[0]);
@@ -161,6 +197,7 @@ __device__ __forceinline__ wf_plan_chunk load_chunk(const wf_plan_chunk* p) {
 
 // ---------------------------------------------------------------- roles
 
+template <bool kFp8>
 __device__ __forceinline__ void producer(const Shared& sh, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                          const CUtensorMap* tm_v, int u0, int u1) {
   int kv_it = 0;
@@ -173,17 +210,30 @@ __device__ __forceinline__ void producer(const Shared& sh, const Params& p, cons
     const bool live1 = p.C - unit.pair * 256 > 128;
     if (q_it > 0 && !wait_bar(sh, p, kBarQEmpty, (q_it - 1) & 1, 1)) { ok = false; break; }
     const uint32_t qbar = smem_u32(sh.bars + kBarQFull);
-    mbar_arrive_expect_tx(qbar, live1 ? 2 * kTileBytes : kTileBytes);
-    tma_load_3d(smem_u32(q_tile(sh, 0)), tm_q, qbar, 0, unit.head, row0);
-    tma_load_3d(smem_u32(q_tile(sh, 0) + kHalfBytes), tm_q, qbar, 64, unit.head, row0);
-    if (live1) {
-      tma_load_3d(smem_u32(q_tile(sh, 1)), tm_q, qbar, 0, unit.head, row0 + 128);
-      tma_load_3d(smem_u32(q_tile(sh, 1) + kHalfBytes), tm_q, qbar, 64, unit.head, row0 + 128);
+    if constexpr (kFp8) {
+      mbar_arrive_expect_tx(qbar, live1 ? 2 * kTile8Bytes : kTile8Bytes);
+      tma_load_3d(smem_u32(q_tile(sh, 0)), tm_q, qbar, 0, unit.head, row0);
+      if (live1) tma_load_3d(smem_u32(q_tile(sh, 1)), tm_q, qbar, 0, unit.head, row0 + 128);
+    } else {
+      mbar_arrive_expect_tx(qbar, live1 ? 2 * kTileBytes : kTileBytes);
+      tma_load_3d(smem_u32(q_tile(sh, 0)), tm_q, qbar, 0, unit.head, row0);
+      tma_load_3d(smem_u32(q_tile(sh, 0) + kHalfBytes), tm_q, qbar, 64, unit.head, row0);
+      if (live1) {
+        tma_load_3d(smem_u32(q_tile(sh, 1)), tm_q, qbar, 0, unit.head, row0 + 128);
+        tma_load_3d(smem_u32(q_tile(sh, 1) + kHalfBytes), tm_q, qbar, 64, unit.head, row0 + 128);
+      }
     }
     ++q_it;
-    for (int j = 0; j < c.key_tiles; ++j) {
+    const int first_slot = kFp8 ? first_visible_slot(p, p.chunks + unit.chunk) : 0;
+    const int n_tiles = unit_key_tiles<kFp8>(p, p.chunks + unit.chunk);
+    for (int j = 0; j < n_tiles; ++j) {
       int32_t tok, valid;
-      key_tile(c, j, tok, valid);
+      if constexpr (kFp8) {
+        int32_t slot, blk;
+        key_tile_fp8(p, first_slot, j, tok, valid, slot, blk);
+      } else {
+        key_tile(c, j, tok, valid);
+      }
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int st = kv_it % kStages;
@@ -195,10 +245,15 @@ __device__ __forceinline__ void producer(const Shared& sh, const Params& p, cons
         }
         if (!wait_bar(sh, p, kBarKVEmpty + st, ((kv_it / kStages) & 1) ^ 1, 2)) { ok = false; break; }
         const uint32_t bar = smem_u32(sh.bars + kBarKVFull + st);
-        mbar_arrive_expect_tx(bar, kTileBytes);
         const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
-        tma_load_3d(smem_u32(kv_tile(sh, st)), tm, bar, 0, unit.head, tok);
-        tma_load_3d(smem_u32(kv_tile(sh, st) + kHalfBytes), tm, bar, 64, unit.head, tok);
+        if (kFp8 && kv == 0) {  // e4m3 K: one 128-byte-wide box
+          mbar_arrive_expect_tx(bar, kTile8Bytes);
+          tma_load_3d(smem_u32(kv_tile(sh, st)), tm, bar, 0, unit.head, tok);
+        } else {
+          mbar_arrive_expect_tx(bar, kTileBytes);
+          tma_load_3d(smem_u32(kv_tile(sh, st)), tm, bar, 0, unit.head, tok);
+          tma_load_3d(smem_u32(kv_tile(sh, st) + kHalfBytes), tm, bar, 64, unit.head, tok);
+        }
         ++kv_it;
       }
       if (!ok) break;
@@ -260,14 +315,26 @@ __device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile) {
   return smem_desc_sw128(smem_u32(tile), kHalfBytes, 1024);
 }
 
+// e4m3 scores: four 32-element K slices, 32 bytes apart inside the 128-byte rows.
+template <int kk>
+__device__ __forceinline__ void issue_s8_slice(uint32_t s_tmem, uint64_t qd, uint64_t kd) {
+  mma_f8_ss_off<kk * 2, kk * 2>(s_tmem, qd, kd, kIdescQK8, kk > 0 ? 1u : 0u);
+  if constexpr (kk < 3) issue_s8_slice<kk + 1>(s_tmem, qd, kd);
+}
+
+template <bool kFp8>
 __device__ __forceinline__ void issue_s(uint32_t s_tmem, uint64_t qd, const uint8_t* k) {
-  issue_s_slice<0>(s_tmem, qd, kmajor_desc(k));
+  if constexpr (kFp8)
+    issue_s8_slice<0>(s_tmem, qd, kmajor_desc(k));
+  else
+    issue_s_slice<0>(s_tmem, qd, kmajor_desc(k));
 }
 
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, const uint8_t* v, bool accumulate) {
   issue_pv_slice<0>(o_tmem, p_tmem, mnmajor_desc(v), accumulate ? 1u : 0u);
 }
 
+template <bool kFp8>
 __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, uint32_t tmem, int u0, int u1) {
   int kv_it = 0, q_it = 0;
   int p_cnt[2] = {0, 0};
@@ -277,7 +344,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
   const uint64_t qd0 = kmajor_desc(q_tile(sh, 0)), qd1 = kmajor_desc(q_tile(sh, 1));
   for (int u = u0; u < u1 && ok; ++u) {
     const wf_plan_unit unit = p.units[u];
-    const int n = __ldg(&p.chunks[unit.chunk].key_tiles);
+    const int n = unit_key_tiles<kFp8>(p, p.chunks + unit.chunk);
     const bool live1 = p.C - unit.pair * 256 > 128;
     if (!wait_bar(sh, p, kBarQFull, q_it & 1, 10)) { ok = false; break; }
     ++q_it;
@@ -286,10 +353,10 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
     if (!wait_bar(sh, p, kBarKVFull + kst, (kv_it / kStages) & 1, 11)) { ok = false; break; }
     ++kv_it;
     tc_fence_after();
-    issue_s(s_tm[0], qd0, kv_tile(sh, kst));
+    issue_s<kFp8>(s_tm[0], qd0, kv_tile(sh, kst));
     mma_commit(smem_u32(sh.bars + kBarSFull + 0));
     if (live1) {
-      issue_s(s_tm[1], qd1, kv_tile(sh, kst));
+      issue_s<kFp8>(s_tm[1], qd1, kv_tile(sh, kst));
       mma_commit(smem_u32(sh.bars + kBarSFull + 1));
     }
     mma_commit(smem_u32(sh.bars + kBarKVEmpty + kst));
@@ -310,7 +377,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
       tc_fence_after();
       issue_pv(o_tm[0], s_tm[0], kv_tile(sh, vst), j > 0);
       if (more) {
-        issue_s(s_tm[0], qd0, kv_tile(sh, kst));
+        issue_s<kFp8>(s_tm[0], qd0, kv_tile(sh, kst));
         mma_commit(smem_u32(sh.bars + kBarSFull + 0));
       } else {
         mma_commit(smem_u32(sh.bars + kBarOFull + 0));
@@ -322,7 +389,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
         tc_fence_after();
         issue_pv(o_tm[1], s_tm[1], kv_tile(sh, vst), j > 0);
         if (more) {
-          issue_s(s_tm[1], qd1, kv_tile(sh, kst));
+          issue_s<kFp8>(s_tm[1], qd1, kv_tile(sh, kst));
           mma_commit(smem_u32(sh.bars + kBarSFull + 1));
         } else {
           mma_commit(smem_u32(sh.bars + kBarOFull + 1));
@@ -341,6 +408,7 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
   }
 }
 
+template <bool kFp8>
 __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, uint32_t tmem, int t, int u0, int u1) {
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -348,18 +416,33 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
   const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
   const uint32_t s_tm = tmem + lane_off + uint32_t(128 * t);
   const uint32_t o_tm = tmem + lane_off + uint32_t(256 + 128 * t);
-  const float sl2 = p.scale_log2;
   int s_cnt = 0, o_cnt = 0;
   for (int u = u0; u < u1; ++u) {
     const wf_plan_unit unit = p.units[u];
     const int rows_here = p.C - unit.pair * 256 - 128 * t;
     if (rows_here <= 0) continue;  // dead tile: the MMA thread skips it too
     const wf_plan_chunk c = load_chunk(p.chunks + unit.chunk);
+    // scores -> log2 units: softmax scale * log2(e), times the query block's
+    // scale on the 8-bit path (the key block's scale is applied per tile)
+    float sl2_unit = p.scale_log2;
+    int first_slot = 0;
+    if constexpr (kFp8) {
+      first_slot = first_visible_slot(p, p.chunks + unit.chunk);
+      sl2_unit *= __ldg(p.q_scales + (int64_t(unit.chunk) * p.nblk + 2 * unit.pair + t) * p.H + unit.head);
+    }
+    const int n_tiles = unit_key_tiles<kFp8>(p, p.chunks + unit.chunk);
     float m_ref = -INFINITY;  // reference max (log2 units)
     float l = 0.f;
-    for (int j = 0; j < c.key_tiles; ++j) {
+    for (int j = 0; j < n_tiles; ++j) {
       int32_t tok, valid;
-      key_tile(c, j, tok, valid);
+      float sl2 = sl2_unit;
+      if constexpr (kFp8) {
+        int32_t slot, blk;
+        key_tile_fp8(p, first_slot, j, tok, valid, slot, blk);
+        sl2 *= __ldg(p.k_scales + (int64_t(slot) * p.nblk + blk) * p.H + unit.head);
+      } else {
+        key_tile(c, j, tok, valid);
+      }
       if (!wait_bar(sh, p, kBarSFull + t, s_cnt & 1, 20 + t)) return;
       ++s_cnt;
       tc_fence_after();
@@ -464,6 +547,7 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
   }
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -498,14 +582,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role(sh, p, tmem, warp / 4, u0, u1);
+    softmax_role<kFp8>(sh, p, tmem, warp / 4, u0, u1);
   } else {
     regs_decrease<kControlRegs>();
     if (warp == 8) {
-      if (lane == 0) mma_issuer(sh, p, tmem, u0, u1);
+      if (lane == 0) mma_issuer<kFp8>(sh, p, tmem, u0, u1);
       __syncwarp();
     } else if (warp == 9 && lane == 0) {
-      producer(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
+      producer<kFp8>(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
     }
   }
   tc_fence_before();
@@ -543,31 +627,34 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// [tokens, H, 128] bf16 viewed as 3-D (dim, head, token); box = 64 dims x 1 head x 128 tokens.
-bool make_tmap(CUtensorMap* tm, const void* base, int64_t tokens, int32_t H) {
+// [tokens, H, 128] viewed as 3-D (dim, head, token).  bf16: box = 64 dims x 1
+// head x 128 tokens (128 bytes wide, loaded as two halves); e4m3 codes: box =
+// all 128 dims (128 bytes) x 1 head x 128 tokens.
+bool make_tmap(CUtensorMap* tm, const void* base, int64_t tokens, int32_t H, bool bytes) {
   auto encode = get_encode();
   if (!encode) return false;
+  const cuuint64_t elem = bytes ? 1 : 2;
   cuuint64_t dims[3] = {128, cuuint64_t(H), cuuint64_t(tokens)};
-  cuuint64_t strides[2] = {128 * 2, cuuint64_t(H) * 128 * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint64_t strides[2] = {128 * elem, cuuint64_t(H) * 128 * elem};
+  cuuint32_t box[3] = {bytes ? 128u : 64u, 1, 128};
   cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = encode(tm, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? true : report("cuTensorMapEncodeTiled", int(r));
 }
 
-}  // namespace
-
-// Launch the tcgen05 path; arguments were validated by the caller.
-wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_rot, const void* k_pool,
-                            const void* v_pool, void* out, float* lse, float scale, void* workspace,
-                            uint64_t timeout_ns, cudaStream_t stream) {
+template <bool kFp8>
+wf_status launch(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q, const float* q_scales,
+                 const void* k_pool, const float* k_scales, const void* v_pool, void* out, float* lse, float scale,
+                 void* workspace, uint64_t timeout_ns, cudaStream_t stream) {
   static int attr_done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WF_ERR_CUDA;
   if (dev < 64 && !attr_done[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const cudaError_t e =
+        cudaFuncSetAttribute(attn_fwd_sm100<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) {
       report(cudaGetErrorString(e), int(e));
       cudaGetLastError();
@@ -576,10 +663,11 @@ wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const
     attr_done[dev] = 1;
   }
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q_rot, int64_t(h->R) * h->C, h->H) || !make_tmap(&tk, k_pool, int64_t(h->S) * h->C, h->H) ||
-      !make_tmap(&tv, v_pool, int64_t(h->S) * h->C, h->H))
+  if (!make_tmap(&tq, q, int64_t(h->R) * h->C, h->H, kFp8) ||
+      !make_tmap(&tk, k_pool, int64_t(h->S) * h->C, h->H, kFp8) ||
+      !make_tmap(&tv, v_pool, int64_t(h->S) * h->C, h->H, false))
     return WF_ERR_CUDA;
-  Params p;
+  Params p{};
   p.chunks = reinterpret_cast<const wf_plan_chunk*>(dev_plan + h->off_chunks);
   p.units = reinterpret_cast<const wf_plan_unit*>(dev_plan + h->off_units);
   p.cta_off = reinterpret_cast<const int32_t*>(dev_plan + h->off_cta);
@@ -593,12 +681,16 @@ wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const
   p.timeout_ns = timeout_ns;
   const char* stall = std::getenv("WF_DEBUG_STALL_FIRST_LOAD");
   p.stall_first_load = (stall && stall[0] == '1') ? 1 : 0;
-  attn_fwd_sm100<<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+  p.q_scales = q_scales;
+  p.k_scales = k_scales;
+  p.S = h->S;
+  p.nblk = (h->C + 127) / 128;
+  attn_fwd_sm100<kFp8><<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     report(cudaGetErrorString(e), int(e));
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_sm100) == cudaSuccess) {
+    if (cudaFuncGetAttributes(&fa, attn_fwd_sm100<kFp8>) == cudaSuccess) {
       char msg[256];
       std::snprintf(msg, sizeof(msg), "attributes: regs %d, max threads %d, static smem %zu, max dyn smem %d",
                     fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.maxDynamicSharedSizeBytes);
@@ -607,6 +699,24 @@ wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const
     return WF_ERR_CUDA;
   }
   return WF_OK;
+}
+
+}  // namespace
+
+// Launch the tcgen05 path; arguments were validated by the caller.
+wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_rot, const void* k_pool,
+                            const void* v_pool, void* out, float* lse, float scale, void* workspace,
+                            uint64_t timeout_ns, cudaStream_t stream) {
+  return launch<false>(h, dev_plan, q_rot, nullptr, k_pool, nullptr, v_pool, out, lse, scale, workspace, timeout_ns,
+                       stream);
+}
+
+// The same with e4m3 Q and K codes and their block scales.
+wf_status launch_attn_sm100_fp8(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q8, const float* q_scales,
+                                const void* k8_pool, const float* k_scales, const void* v_pool, void* out, float* lse,
+                                float scale, void* workspace, uint64_t timeout_ns, cudaStream_t stream) {
+  return launch<true>(h, dev_plan, q8, q_scales, k8_pool, k_scales, v_pool, out, lse, scale, workspace, timeout_ns,
+                      stream);
 }
 
 }  // namespace wf

@@ -157,6 +157,20 @@ __device__ __forceinline__ void mma_ss_off(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// The same with e4m3 operands (kind::f8f6f4: 32 K elements per instruction).
+template <uint32_t kAOff, uint32_t kBOff>
+__device__ __forceinline__ void mma_f8_ss_off(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "add.s64 da, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kAOff), "n"(kBOff)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem + kACol] * B[smem desc + kBOff].
 template <uint32_t kACol, uint32_t kBOff>
 __device__ __forceinline__ void mma_ts_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -248,6 +262,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo
 //   [15] A major (0 = K); [16] B major (1 = MN); [17,23) N>>3; [24,29) M>>4.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32, A and B e4m3 (format 0),
+// both K-major, dense.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
+  return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -96,7 +96,8 @@ class Rollout:
     """Device state of one stream: the K/V ring pool, the round's buffers, plan and workspace."""
 
     def __init__(self, cfg: RoundConfig, device="cuda", seed: int = 42, first_n0: Optional[int] = None,
-                 num_ctas: int = 0, want_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):
+                 num_ctas: int = 0, want_lse: bool = True, stream: Optional[torch.cuda.Stream] = None,
+                 fp8: bool = False):
         self.cfg = cfg
         self.device = torch.device(device)
         self.seed = seed
@@ -115,6 +116,16 @@ class Rollout:
         self.q_rot = torch.empty(nq, H, D, **kw)
         self.out = torch.empty(nq, H, D, **kw)
         self.lse = torch.empty(H, nq, dtype=torch.float32, device=self.device) if want_lse else None
+        # 8-bit scores: e4m3 codes of Q' and of the pool's K' with their block scales
+        self.fp8 = fp8
+        if fp8:
+            if cfg.dtype != wf.WF_BF16:
+                raise ValueError("the 8-bit score path takes bf16 rounds")
+            nblk = -(-C // wf.WF_FP8_BLOCK)
+            self.q8 = torch.empty(nq, H, D, dtype=torch.uint8, device=self.device)
+            self.q_scales = torch.empty(max(R, 1), nblk, H, dtype=torch.float32, device=self.device)
+            self.k8_pool = torch.zeros(S * C, H, D, dtype=torch.uint8, device=self.device)
+            self.k_scales = torch.ones(S, nblk, H, dtype=torch.float32, device=self.device)
         self._plan_cap = 0
         self._ensure_plan_capacity(wf.wf_plan_bytes(self.desc(self.first_n0)))
         self.workspace = torch.empty(4096, dtype=torch.uint8, device=self.device)
@@ -167,6 +178,8 @@ class Rollout:
             self._plan(self.desc(n, R=g, Wc=0, noise=[0] * g))
             wf.wf_rope3d_append(self.host_plan, self.dev_plan, self.q, self.k, self.v, self.q_rot, self.k_pool,
                                 self.v_pool, self.stream)
+            if self.fp8:
+                wf.wf_quantize_fp8(self.host_plan, self.k_pool, self.k8_pool, self.k_scales, wf.WF_FP8_K, self.stream)
             n += g
         self.round_index = -1
 
@@ -180,10 +193,22 @@ class Rollout:
     def append(self):
         wf.wf_rope3d_append(self.host_plan, self.dev_plan, self.q, self.k, self.v, self.q_rot, self.k_pool,
                             self.v_pool, self.stream)
+        if self.fp8:
+            self.quantize()
+
+    def quantize(self):
+        """e4m3 codes and block scales of this round's Q' and of its chunks' K' in the pool."""
+        wf.wf_quantize_fp8(self.host_plan, self.q_rot, self.q8, self.q_scales, wf.WF_FP8_Q, self.stream)
+        wf.wf_quantize_fp8(self.host_plan, self.k_pool, self.k8_pool, self.k_scales, wf.WF_FP8_K, self.stream)
 
     def attend(self, scale: float = 0.0):
-        wf.wf_chunk_causal_attn(self.host_plan, self.dev_plan, self.q_rot, self.k_pool, self.v_pool, self.out,
-                                self.lse, scale, self.workspace, self.stream)
+        if self.fp8:
+            wf.wf_chunk_causal_attn_fp8(self.host_plan, self.dev_plan, self.q8, self.q_scales, self.k8_pool,
+                                        self.k_scales, self.v_pool, self.out, self.lse, scale, self.workspace,
+                                        self.stream)
+        else:
+            wf.wf_chunk_causal_attn(self.host_plan, self.dev_plan, self.q_rot, self.k_pool, self.v_pool, self.out,
+                                    self.lse, scale, self.workspace, self.stream)
 
     def run_round(self, r: int, fill: bool = True):
         """Generate round r's inputs (tag r), plan, RoPE/append, attention."""
@@ -206,19 +231,25 @@ class Rollout:
         resuming is restoring the pool and planning the next round.
         """
         self.stream.synchronize()
-        return {"round": self.round_index, "first_n0": self.first_n0, "seed": self.seed,
-                "k_pool": self.k_pool.cpu(), "v_pool": self.v_pool.cpu()}
+        state = {"round": self.round_index, "first_n0": self.first_n0, "seed": self.seed,
+                 "k_pool": self.k_pool.cpu(), "v_pool": self.v_pool.cpu()}
+        if self.fp8:
+            state.update(k8_pool=self.k8_pool.cpu(), k_scales=self.k_scales.cpu())
+        return state
 
     def restore(self, state: dict):
         """Load a checkpoint() taken from a rollout of the same configuration."""
-        for name in ("k_pool", "v_pool"):
+        names = ("k_pool", "v_pool") + (("k8_pool", "k_scales") if self.fp8 else ())
+        for name in names:
+            if name not in state:
+                raise ValueError(f"checkpoint has no {name}")
             src, dst = state[name], getattr(self, name)
             if src.shape != dst.shape or src.dtype != dst.dtype:
                 raise ValueError(f"checkpoint {name} is {tuple(src.shape)} {src.dtype}, "
                                  f"this rollout holds {tuple(dst.shape)} {dst.dtype}")
         with torch.cuda.stream(self.stream):
-            self.k_pool.copy_(state["k_pool"], non_blocking=False)
-            self.v_pool.copy_(state["v_pool"], non_blocking=False)
+            for name in names:
+                getattr(self, name).copy_(state[name], non_blocking=False)
         self.first_n0 = int(state["first_n0"])
         self.seed = int(state["seed"])
         self.round_index = int(state["round"])

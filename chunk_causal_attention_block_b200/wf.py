@@ -24,11 +24,14 @@ WF_OK, WF_ERR_INVALID_ARG, WF_ERR_UNSUPPORTED, WF_ERR_ALIGNMENT, WF_ERR_CAPACITY
 WF_F32, WF_BF16 = 0, 1
 WF_MAX_INROUND = 16
 WF_SYNTH_Q, WF_SYNTH_K, WF_SYNTH_V = 1, 2, 3
+WF_FP8_BLOCK = 128
+WF_FP8_Q, WF_FP8_K = 0, 1
 
 # exported symbols, in the order include/wf.h and include/wf_synth.h declare them
 EXPORTS = ("wf_plan_bytes", "wf_plan_round", "wf_rope3d_append", "wf_attn_workspace_bytes",
            "wf_attn_workspace_init", "wf_attn_workspace_status", "wf_chunk_causal_attn",
-           "wf_chunk_causal_attn_noalloc", "wf_status_string", "wf_version", "wf_synth_fill")
+           "wf_chunk_causal_attn_noalloc", "wf_quantize_fp8", "wf_chunk_causal_attn_fp8", "wf_status_string",
+           "wf_version", "wf_synth_fill")
 
 
 class WfError(RuntimeError):
@@ -86,6 +89,9 @@ def lib() -> ctypes.CDLL:
         L.wf_chunk_causal_attn.restype = i32
         L.wf_chunk_causal_attn_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp]
         L.wf_chunk_causal_attn_noalloc.restype = i32
+        L.wf_quantize_fp8.argtypes, L.wf_quantize_fp8.restype = [vp, vp, vp, vp, i32, vp], i32
+        L.wf_chunk_causal_attn_fp8.argtypes = [vp] * 9 + [ctypes.c_float, vp, sz, vp]
+        L.wf_chunk_causal_attn_fp8.restype = i32
         L.wf_status_string.argtypes, L.wf_status_string.restype = [i32], ctypes.c_char_p
         L.wf_version.argtypes, L.wf_version.restype = [], i32
         L.wf_synth_fill.argtypes = [vp, i32, u64, i32, i64, i64, i32, i32, i32, i32, i32, vp]
@@ -175,6 +181,19 @@ def wf_chunk_causal_attn_noalloc(host_plan, dev_plan, q_rot, k_pool, v_pool, out
                                               _ptr(v_pool), _ptr(out), _ptr(lse), float(softmax_scale),
                                               _stream(stream)), "wf_chunk_causal_attn_noalloc")
 
+
+
+def wf_quantize_fp8(host_plan, src, dst8, scales, which, stream=None):
+    _check(lib().wf_quantize_fp8(_ptr(host_plan), _ptr(src), _ptr(dst8), _ptr(scales), int(which), _stream(stream)),
+           "wf_quantize_fp8")
+
+
+def wf_chunk_causal_attn_fp8(host_plan, dev_plan, q8, q_scales, k8_pool, k_scales, v_pool, out, lse=None,
+                             softmax_scale=0.0, workspace=None, stream=None, workspace_bytes=None):
+    wb = workspace_bytes if workspace_bytes is not None else _nbytes(workspace)
+    _check(lib().wf_chunk_causal_attn_fp8(_ptr(host_plan), _ptr(dev_plan), _ptr(q8), _ptr(q_scales), _ptr(k8_pool),
+                                          _ptr(k_scales), _ptr(v_pool), _ptr(out), _ptr(lse), float(softmax_scale),
+                                          _ptr(workspace), wb, _stream(stream)), "wf_chunk_causal_attn_fp8")
 
 def wf_synth_fill(dst, dtype, seed, tensor, tag, n_first, nchunks, C, H, D, kscale=False, stream=None):
     _check(lib().wf_synth_fill(_ptr(dst), int(dtype), int(seed) & 0xFFFFFFFFFFFFFFFF, int(tensor), int(tag),

@@ -222,6 +222,57 @@ wf_status wf_chunk_causal_attn_noalloc(const void* host_plan, const void* dev_pl
                                        const void* q_rot, const void* k_pool, const void* v_pool,
                                        void* out, float* lse, float softmax_scale, wf_stream_t stream);
 
+/*
+ * 8-bit scores.  The Wave Forcing abstract (arXiv 2611.00859v1) measures its
+ * system with 8-bit attention backends; these two calls are this library's
+ * B200 counterpart: Q' and K' as OCP FP8 E4M3 codes with one fp32 scale per
+ * block, scores on the tensor cores' e4m3 path (kind::f8f6f4), P and V in
+ * bf16 as in wf_chunk_causal_attn.
+ *
+ * Blocks are WF_FP8_BLOCK consecutive tokens of one chunk (chunk-relative,
+ * the last one ragged: nblk = ceil(C / WF_FP8_BLOCK) per chunk) times one
+ * head.  scale = amax / 448 in fp32 (1 for an all-zero block) and each
+ * element becomes the e4m3 value nearest x / scale (one fp32 division, then
+ * nearest-even conversion that saturates at +-448).
+ */
+#define WF_FP8_BLOCK 128
+typedef enum wf_fp8_which { WF_FP8_Q = 0, WF_FP8_K = 1 } wf_fp8_which;
+
+/*
+ * wf_quantize_fp8 -- e4m3 codes and block scales of the round's rotated
+ * queries (WF_FP8_Q) or of the in-round chunks' rotated keys in the pool
+ * (WF_FP8_K).  Run it after wf_rope3d_append of the same round; the cache
+ * chunks keep the codes written in their last in-round round.
+ *
+ * WF_FP8_Q: src = q_rot [R*C, H, D] bf16; dst8 = [R*C, H, D] bytes;
+ *           scales = [R, nblk, H] fp32.
+ * WF_FP8_K: src = k_pool [S*C, H, D] bf16; dst8 = [S*C, H, D] bytes (only the
+ *           in-round slots are written); scales = [S, nblk, H] fp32 (only the
+ *           in-round slots' rows).
+ * Requires a bf16 plan with D = 128; pointers 16-byte aligned (scales 4).
+ * Errors: WF_ERR_INVALID_ARG, WF_ERR_PLAN, WF_ERR_ALIGNMENT,
+ *         WF_ERR_UNSUPPORTED, WF_ERR_CUDA.
+ */
+wf_status wf_quantize_fp8(const void* host_plan, const void* src, void* dst8, float* scales, int32_t which,
+                          wf_stream_t stream);
+
+/*
+ * wf_chunk_causal_attn_fp8 -- wf_chunk_causal_attn with the scores computed
+ * from the e4m3 codes: S = (q8 k8^T) * q_scale * k_scale per (query block,
+ * key block), then the same online softmax, bf16 P and PV with bf16 V.  The
+ * key tiles are the chunks' scale blocks (each visible chunk is walked on
+ * its own, nblk tiles, the last one ragged).
+ *
+ * q8, q_scales: from wf_quantize_fp8(WF_FP8_Q); k8_pool, k_scales: from
+ * wf_quantize_fp8(WF_FP8_K) over the stream so far; v_pool, out, lse,
+ * softmax_scale, workspace as in wf_chunk_causal_attn.
+ * Errors: as wf_chunk_causal_attn (bf16 plans with D = 128 only).
+ */
+wf_status wf_chunk_causal_attn_fp8(const void* host_plan, const void* dev_plan, const void* q8,
+                                   const float* q_scales, const void* k8_pool, const float* k_scales,
+                                   const void* v_pool, void* out, float* lse, float softmax_scale,
+                                   void* workspace, size_t workspace_bytes, wf_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* wf_status_string(wf_status status);
 

@@ -50,15 +50,15 @@ def oracle_inputs(cfg: RoundConfig, n0: int, first_n0: int, heads, seed=42, k_ov
     return q, k, v, kc, vc
 
 
-def oracle_call(cfg: RoundConfig, n0: int, arrays, rows=None):
+def oracle_call(cfg: RoundConfig, n0: int, arrays, rows=None, fp8=False):
     q, k, v, kc, vc = arrays
     return orc.wave_round(q, k, v, kc, vc, n0=n0, F=cfg.F, fh=cfg.fh, fw=cfg.fw, pairs=pairs_of(cfg),
-                          theta=cfg.theta, dtype=dtype_name(cfg), rows=rows)
+                          theta=cfg.theta, dtype=dtype_name(cfg), rows=rows, fp8=fp8)
 
 
-def oracle_round(cfg: RoundConfig, n0: int, first_n0: int, heads, rows=None, seed=42, k_override=None):
+def oracle_round(cfg: RoundConfig, n0: int, first_n0: int, heads, rows=None, seed=42, k_override=None, fp8=False):
     """Oracle result of the round with oldest in-round chunk n0, restricted to `heads`."""
-    return oracle_call(cfg, n0, oracle_inputs(cfg, n0, first_n0, heads, seed, k_override), rows)
+    return oracle_call(cfg, n0, oracle_inputs(cfg, n0, first_n0, heads, seed, k_override), rows, fp8)
 
 
 def sample_rows(cfg: RoundConfig, extra=24, seed=0):
@@ -98,9 +98,9 @@ def assert_f32_close(got, want, what=""):
         assert rel <= F32_REL, f"{what} head {h}: {rel}"
 
 
-def run_rollout(cfg: RoundConfig, rounds, first_n0=None, num_ctas=0, seed=42, on_round=None):
+def run_rollout(cfg: RoundConfig, rounds, first_n0=None, num_ctas=0, seed=42, on_round=None, fp8=False):
     """Prefill, then run rounds 0..max(rounds); call on_round(ro, r) after each listed round."""
-    ro = Rollout(cfg, seed=seed, first_n0=first_n0, num_ctas=num_ctas)
+    ro = Rollout(cfg, seed=seed, first_n0=first_n0, num_ctas=num_ctas, fp8=fp8)
     ro.prefill()
     last = max(rounds)
     for r in range(last + 1):
@@ -114,9 +114,10 @@ def run_rollout(cfg: RoundConfig, rounds, first_n0=None, num_ctas=0, seed=42, on
     return ro
 
 
-def check_attention(ro: Rollout, r: int, heads, rows, what=""):
+def check_attention(ro: Rollout, r: int, heads, rows, what="", fp8=None):
     cfg = ro.cfg
-    ref = oracle_round(cfg, ro.n0_of(r), ro.first_n0, heads, rows=rows, seed=ro.seed)
+    fp8 = ro.fp8 if fp8 is None else fp8
+    ref = oracle_round(cfg, ro.n0_of(r), ro.first_n0, heads, rows=rows, seed=ro.seed, fp8=fp8)
     got = to_np(ro.out[rows][:, heads])
     if cfg.dtype == wf.WF_BF16:
         e = assert_bf16_close(got, ref["O"], what)

@@ -118,6 +118,31 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
     assert wf.wf_attn_workspace_bytes(bad) == 0
 
 
+def test_fp8_entry_points_reject_bad_arguments_before_any_launch():
+    f32 = _plan(_desc())
+    bf16 = _plan(_desc(D=128, dtype=wf.WF_BF16))
+    fake = 1 << 20  # never dereferenced: validation fails first
+    cases = [
+        (lambda: wf.wf_quantize_fp8(f32, fake, fake, fake, wf.WF_FP8_K), wf.WF_ERR_UNSUPPORTED),
+        (lambda: wf.wf_quantize_fp8(bf16, fake, fake, fake, 2), wf.WF_ERR_INVALID_ARG),
+        (lambda: wf.wf_quantize_fp8(bf16, fake, fake, None, wf.WF_FP8_Q), wf.WF_ERR_INVALID_ARG),
+        (lambda: wf.wf_quantize_fp8(bf16, fake + 8, fake, fake, wf.WF_FP8_Q), wf.WF_ERR_ALIGNMENT),
+        (lambda: wf.wf_quantize_fp8(bf16, fake, fake, fake + 2, wf.WF_FP8_Q), wf.WF_ERR_ALIGNMENT),
+        (lambda: wf.wf_chunk_causal_attn_fp8(bf16, fake, fake, fake, fake, fake, fake, fake, None, 0.0, fake,
+                                             workspace_bytes=16), wf.WF_ERR_WORKSPACE),
+        (lambda: wf.wf_chunk_causal_attn_fp8(bf16, fake, fake, fake, fake, None, fake, fake, None, 0.0, fake,
+                                             workspace_bytes=4096), wf.WF_ERR_INVALID_ARG),
+        (lambda: wf.wf_chunk_causal_attn_fp8(bf16, fake, fake, fake + 2, fake, fake, fake, fake, None, 0.0, fake,
+                                             workspace_bytes=4096), wf.WF_ERR_ALIGNMENT),
+        (lambda: wf.wf_chunk_causal_attn_fp8(f32, fake, fake, fake, fake, fake, fake, fake, None, 0.0, fake,
+                                             workspace_bytes=4096), wf.WF_ERR_UNSUPPORTED),
+    ]
+    for call, code in cases:
+        with pytest.raises(wf.WfError) as e:
+            call()
+        assert e.value.code == code
+
+
 def _compare_plan(host, ref, desc_kw):
     p = wf.decode_plan(host)
     assert p["magic"] == 0x31504657 and p["version"] == 1

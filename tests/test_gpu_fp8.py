@@ -1,0 +1,116 @@
+"""8-bit score path on the GPU, through the C ABI, against the oracle.
+
+Bit-exact: the e4m3 codes and fp32 block scales of Q' and of the pool's K'
+(wf_quantize_fp8) against the oracle's fp8_block_quantize.  Within the bf16
+gates (max-abs 2e-2, mean-abs 2e-3, relative RMS 1e-2): the attention of
+wf_chunk_causal_attn_fp8 against the oracle evaluated on the same
+dequantized codes.  Accuracy of the variant itself: against the exact
+(16-bit input) oracle the stated gates still hold and the relative RMS error
+stays below 6e-2 (e4m3 keeps 3 mantissa bits: a relative rounding error of at
+most 2^-4 per element of Q and K; the oracle alone measures about 3.9e-2 on
+these inputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+from chunk_causal_attention_block_b200 import wf
+from chunk_causal_attention_block_b200.rollout import CONFIGS, RoundConfig
+from tests import gpu_common as gc
+
+pytestmark = pytest.mark.gpu
+
+FP8_VS_EXACT_REL_RMS = 6e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    wf.lib()
+    yield
+
+
+def _e4m3_values(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
+
+
+def _check_codes(ro, r, heads):
+    cfg = ro.cfg
+    n0 = ro.n0_of(r)
+    ref = gc.oracle_round(cfg, n0, ro.first_n0, heads, rows=np.array([0]), seed=ro.seed, fp8=True)
+    C, S, R = cfg.C, cfg.slots, cfg.R
+    q8 = _e4m3_values(ro.q8[:R * C][:, heads])
+    assert np.array_equal(q8, ref["q8"]), "Q codes"
+    assert np.array_equal(ro.q_scales[:R][:, :, heads].cpu().numpy().astype(np.float64), ref["q_scales"]), "Q scales"
+    wc_eff = min(cfg.Wc, n0)
+    k8 = _e4m3_values(ro.k8_pool.view(S, C, cfg.H, cfg.D)[:, :, heads])
+    ks = ro.k_scales[:, :, heads].cpu().numpy().astype(np.float64)
+    chunks = list(range(n0 - wc_eff, n0 + R))
+    got_k8 = np.concatenate([k8[n % S] for n in chunks])
+    got_ks = np.stack([ks[n % S] for n in chunks])
+    assert np.array_equal(got_k8, ref["k8"]), "K codes"
+    assert np.array_equal(got_ks, ref["k_scales"]), "K scales"
+
+
+SMALL = [
+    RoundConfig("ragged small", H=2, D=128, fh=10, fw=10, F=3, Wc=3, R=3, noise_t=(250, 500, 750)),
+    RoundConfig("tiny chunks", H=3, D=128, fh=5, fw=7, F=2, Wc=2, R=4, noise_t=(0, 250, 500, 750)),
+    RoundConfig("C=1", H=2, D=128, fh=1, fw=1, F=1, Wc=5, R=4, noise_t=(250, 500, 750, 1000)),
+    RoundConfig("no cache", H=2, D=128, fh=9, fw=13, F=2, Wc=0, R=1, noise_t=(1000,)),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_fp8_codes_bit_exact_and_attention_all_rows(cfg):
+    rows = np.arange(cfg.R * cfg.C)
+    heads = list(range(cfg.H))
+
+    def on_round(ro, r):
+        _check_codes(ro, r, heads)
+        gc.check_attention(ro, r, heads, rows, f"{cfg.name} r{r}")
+
+    gc.run_rollout(cfg, (0, 1, cfg.Wc + cfg.R + 1), on_round=on_round, fp8=True)
+
+
+@pytest.mark.parametrize("name,heads,rounds", [("wan13b_round", [2, 9], (0, 7)), ("wan14b_round", [5, 33], (0,))])
+def test_fp8_full_size_sampled(name, heads, rounds):
+    cfg = CONFIGS[name]
+    rows = gc.sample_rows(cfg, extra=12)
+
+    def on_round(ro, r):
+        _check_codes(ro, r, heads[:1])
+        gc.check_attention(ro, r, heads, rows, f"{name} r{r}")
+
+    gc.run_rollout(cfg, rounds, on_round=on_round, fp8=True)
+
+
+def test_fp8_accuracy_against_the_exact_oracle():
+    cfg = CONFIGS["wan13b_round"]
+    rows = gc.sample_rows(cfg, extra=12)
+    errs = []
+
+    def on_round(ro, r):
+        ref = gc.oracle_round(cfg, ro.n0_of(r), ro.first_n0, [4], rows=rows, seed=ro.seed)
+        got = gc.to_np(ro.out[rows][:, [4]])
+        errs.append(gc.bf16_errors(got, ref["O"]))
+
+    gc.run_rollout(cfg, (0,), on_round=on_round, fp8=True)
+    e = errs[0]
+    assert e["max_abs"] <= 2e-2 and e["mean_abs"] <= 2e-3, e
+    assert e["rel_rms"] <= FP8_VS_EXACT_REL_RMS, e
+
+
+def test_fp8_rollout_resumes_bit_identically():
+    cfg = SMALL[0]
+    a = gc.run_rollout(cfg, (3,), fp8=True)
+    state = a.checkpoint()
+    a.run_round(4)
+    torch.cuda.synchronize()
+    want = a.out.clone()
+    from chunk_causal_attention_block_b200.rollout import Rollout
+    b = Rollout(cfg, fp8=True)
+    b.restore(state)
+    b.run_round(4)
+    torch.cuda.synchronize()
+    assert torch.equal(b.out, want)
