@@ -8,9 +8,12 @@
 // threads takes sixteen rows per pass and keeps its eight passes in
 // registers while the block's absolute maximum is reduced, then writes the
 // codes (8 bytes per thread per row) and the block scale.
-//   scale = amax / 448 (fp32, nearest; 1 for an all-zero block)
-//   code  = e4m3(x / scale): one fp32 division, then the nearest-even
-//           conversion that saturates at +-448.
+//   scale = amax / 448 and inv = 448 / amax (fp32, nearest; both 1 for an
+//           all-zero block)
+//   code  = e4m3(x * inv): one fp32 product, then the nearest-even
+//           conversion that saturates at +-448.  (A product instead of a
+//           division by scale: the correctly rounded division made the
+//           kernel instruction-bound.)
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -46,11 +49,11 @@ __device__ __forceinline__ float abs_max8(const uint4& v, float m) {
   return m;
 }
 
-__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d, float scale) {
-  const uint32_t qa = __nv_cvt_float_to_fp8(__fdiv_rn(a, scale), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t qb = __nv_cvt_float_to_fp8(__fdiv_rn(b, scale), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t qc = __nv_cvt_float_to_fp8(__fdiv_rn(c, scale), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t qd = __nv_cvt_float_to_fp8(__fdiv_rn(d, scale), __NV_SATFINITE, __NV_E4M3);
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d, float inv) {
+  const uint32_t qa = __nv_cvt_float_to_fp8(__fmul_rn(a, inv), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t qb = __nv_cvt_float_to_fp8(__fmul_rn(b, inv), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t qc = __nv_cvt_float_to_fp8(__fmul_rn(c, inv), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t qd = __nv_cvt_float_to_fp8(__fmul_rn(d, inv), __NV_SATFINITE, __NV_E4M3);
   return qa | (qb << 8) | (qc << 16) | (qd << 24);  // lowest address = lowest dim
 }
 
@@ -80,6 +83,7 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const QuantParams p) {
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
   const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
 #pragma unroll
   for (int s = 0; s < kPasses; ++s) {
     const int r = s * kRowsPerPass + r0;
@@ -88,8 +92,8 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const QuantParams p) {
       const float2 f0 = __bfloat1622float2(x[0]), f1 = __bfloat1622float2(x[1]);
       const float2 f2 = __bfloat1622float2(x[2]), f3 = __bfloat1622float2(x[3]);
       uint2 q;
-      q.x = e4m3x4(f0.x, f0.y, f1.x, f1.y, scale);
-      q.y = e4m3x4(f2.x, f2.y, f3.x, f3.y, scale);
+      q.x = e4m3x4(f0.x, f0.y, f1.x, f1.y, inv);
+      q.y = e4m3x4(f2.x, f2.y, f3.x, f3.y, inv);
       p.dst[((tok0 + r) * p.H + h) * 16 + part] = q;
     }
   }

@@ -231,9 +231,10 @@ wf_status wf_chunk_causal_attn_noalloc(const void* host_plan, const void* dev_pl
  *
  * Blocks are WF_FP8_BLOCK consecutive tokens of one chunk (chunk-relative,
  * the last one ragged: nblk = ceil(C / WF_FP8_BLOCK) per chunk) times one
- * head.  scale = amax / 448 in fp32 (1 for an all-zero block) and each
- * element becomes the e4m3 value nearest x / scale (one fp32 division, then
- * nearest-even conversion that saturates at +-448).
+ * head.  scale = amax / 448 and inv = 448 / amax in fp32 (both 1 for an
+ * all-zero block); each element becomes the e4m3 value nearest x * inv (one
+ * fp32 product, then the nearest-even conversion that saturates at +-448),
+ * and is read back as code * scale.
  */
 #define WF_FP8_BLOCK 128
 typedef enum wf_fp8_which { WF_FP8_Q = 0, WF_FP8_K = 1 } wf_fp8_which;

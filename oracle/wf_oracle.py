@@ -290,8 +290,8 @@ def attention_bruteforce(q, k, v, mask, scale: float):
 # attention backends the Wave Forcing abstract benchmarks against) quantizes
 # the rotated Q and K, not V: per (chunk, block of FP8_BLOCK consecutive
 # chunk-relative tokens, head) one fp32 scale = amax / 448, and every element
-# becomes the e4m3 value nearest x / scale.  Scores are products of the
-# dequantized values; P and V stay as in the 16-bit path.
+# becomes the e4m3 value nearest x * (448 / amax).  Scores are products of
+# the dequantized values (code * scale); P and V stay as in the 16-bit path.
 
 E4M3_MAX = 448.0   # largest finite e4m3 value (1.75 * 2^8)
 FP8_BLOCK = 128    # tokens per scale block
@@ -314,10 +314,10 @@ def fp8_block_quantize(x, C: int):
     """x: [n*C, H, D] values (exact in fp32), n whole chunks of C tokens.
 
     Per chunk, block b of tokens [b*FP8_BLOCK, min(C, (b+1)*FP8_BLOCK)) and
-    head: scale = fp32(amax / 448) (1 for an all-zero block), codes =
-    round_e4m3(fp32(x / scale)).  Both divisions are single fp32 divisions
-    rounded to nearest.  Returns (codes [n*C, H, D] as values, scales
-    [n, nblk, H] float64 holding fp32 values).
+    head: scale = fp32(amax / 448), inv = fp32(448 / amax) (both 1 for an
+    all-zero block), codes = round_e4m3(fp32(x * inv)).  Every fp32
+    operation is a single operation rounded to nearest.  Returns (codes
+    [n*C, H, D] as values, scales [n, nblk, H] float64 holding fp32 values).
     """
     x = np.asarray(x, dtype=np.float64)
     T, H, D = x.shape
@@ -330,9 +330,12 @@ def fp8_block_quantize(x, C: int):
             lo, hi = c * C + b * FP8_BLOCK, c * C + min(C, (b + 1) * FP8_BLOCK)
             blk = x[lo:hi].astype(np.float32)                       # [tokens, H, D], exact
             amax = np.abs(blk).max(axis=(0, 2))                      # [H]
-            sc = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+            nz = amax > 0
+            safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+            sc = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+            inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
             scales[c, b] = sc
-            codes[lo:hi] = round_e4m3((blk / sc[None, :, None]).astype(np.float32))
+            codes[lo:hi] = round_e4m3((blk * inv[None, :, None]).astype(np.float32))
     return codes, scales
 
 

@@ -414,7 +414,7 @@ def test_fp8_block_quantize_hand_case():
     assert np.array_equal(codes[5, 0], [448.0, -128.0, 32.0, 0.0])   # x * 128, all representable
     assert np.array_equal(codes[70, 0], [-256.0, 192.0, 0.0, 16.0])
     assert abs(codes[129, 0, 0]) == 448.0                             # the block max maps to the largest code
-    assert codes[129, 0, 3] == orc.round_e4m3(np.float32(-0.375) / np.float32(scales[0, 1, 0]))
+    assert codes[129, 0, 3] == orc.round_e4m3(np.float32(-0.375) * (np.float32(448.0) / np.float32(0.75)))
     assert not codes[:, 1].any()
     deq = orc.fp8_dequantize(codes, scales, C)
     assert np.array_equal(deq[5, 0], x[5, 0]) and np.array_equal(deq[70, 0], x[70, 0])
@@ -430,7 +430,7 @@ def test_fp8_dequantized_error_within_half_an_e4m3_step():
     tok = np.arange(2 * C)
     sc = scales[tok // C, (tok % C) // orc.FP8_BLOCK][:, :, None]
     # half a step of the binade (relative 2^-4) for normals, 2^-10 * scale in the subnormal range,
-    # plus the fp32 rounding of x / scale (relative 2^-24)
+    # plus the fp32 roundings of 448 / amax, amax / 448 and x * inv (relative 2^-24 each)
     bound = np.maximum(np.abs(x) * 2.0 ** -4, sc * 2.0 ** -10) * (1 + 2.0 ** -20)
     assert (np.abs(deq - x) <= bound).all()
 
