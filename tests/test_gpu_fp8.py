@@ -114,3 +114,19 @@ def test_fp8_rollout_resumes_bit_identically():
     b.run_round(4)
     torch.cuda.synchronize()
     assert torch.equal(b.out, want)
+
+
+def test_fp8_stream_start_and_refresh_round():
+    # a stream that starts with one clean chunk (the window grows round by round)
+    cfg = SMALL[0]
+    rows = np.arange(cfg.R * cfg.C)
+
+    def on_round(ro, r):
+        _check_codes(ro, r, [0, 1])
+        gc.check_attention(ro, r, [0, 1], rows, f"start r{r}")
+
+    gc.run_rollout(cfg, (0, 1, 2, 4), first_n0=1, on_round=on_round, fp8=True)
+    # a cache-refresh round at full size (t = 0 member first)
+    ref_cfg = CONFIGS["wan13b_refresh"]
+    srows = gc.sample_rows(ref_cfg, extra=8)
+    gc.run_rollout(ref_cfg, (0,), on_round=lambda ro, r: gc.check_attention(ro, r, [6], srows, "refresh"), fp8=True)
