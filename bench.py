@@ -60,11 +60,20 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_sha():
+def kernel_source_sha(read=None):
+    """Hash of the attention kernel's code (line comments and blank lines
+    dropped, so that editing a comment does not orphan a capture)."""
     h = hashlib.sha256()
     for name in ("attn_sm100.cu", "sm100_ptx.cuh", "wf_plan.h", "wf_plan.cpp"):
-        with open(os.path.join(ROOT, "chunk_causal_attention_block_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, "chunk_causal_attention_block_b200", "csrc", name)) as f:
+                text = f.read()
+        else:
+            text = read(name)
+        for line in text.splitlines():
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

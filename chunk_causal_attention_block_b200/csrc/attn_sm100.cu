@@ -32,6 +32,13 @@
 // below 256 and the fp32 sums stay exact enough; the final O / l uses the
 // same reference, so the result is unchanged.
 //
+// The kFp8 instantiation computes the scores from e4m3 codes: Q and K tiles
+// are 128 rows x 128 bytes (one TMA box each), S_t is four kind::f8f6f4 MMAs
+// of 32 K elements, and the key tiles are the chunks' 128-token scale blocks
+// (each visible chunk walked on its own, its last tile ragged), so that the
+// softmax scales a tile's scores by one factor, q_scale * k_scale.  P, V, O
+// and everything else are as in the bf16 instantiation.
+//
 // Every mbarrier wait is bounded by a time limit; on expiry the CTA records
 // WF_ERR_DEVICE_TIMEOUT in the workspace status word, stops issuing work,
 // drains what it issued and frees its TMEM before returning.
