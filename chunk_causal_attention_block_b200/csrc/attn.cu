@@ -9,6 +9,7 @@
 // partial dot products are summed with warp shuffles.  K/V tiles of 32 keys
 // are staged in shared memory and the online softmax is updated once per
 // tile.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -114,6 +115,82 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const F32Params p) {
 
 bool misaligned(const void* ptr) { return reinterpret_cast<uintptr_t>(ptr) % 16 != 0; }
 
+// Units whose keys the plan split into parts leave normalised partial O and
+// LSE rows in the workspace; this pass merges the parts of every (chunk,
+// head, row pair): LSE = log sum_k exp(LSE_k), O = sum_k exp(LSE_k - LSE) O_k.
+// One warp per row, four dims per lane; a block covers 8 rows of one pair.
+struct CombineParams {
+  const float* part_o;    // [units][256][128]
+  const float* part_lse;  // [units][256]
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t H, C, q_pairs, parts, rc;
+};
+
+__global__ void __launch_bounds__(256) attn_combine_kernel(const CombineParams p) {
+  const int g = blockIdx.x;  // (chunk, head, row pair); its parts are slots g*parts .. g*parts+parts-1
+  const int pair = g % p.q_pairs, ih = g / p.q_pairs, h = ih % p.H, i = ih / p.H;
+  const int rows = min(256, p.C - pair * 256);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y * 8 + warp;
+  if (r < rows) {
+    const float lk = lane < p.parts ? p.part_lse[(int64_t(g) * p.parts + lane) * 256 + r] : -INFINITY;
+    float mx = lk;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float w = lane < p.parts ? expf(lk - mx) : 0.f;
+    float wsum = w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < p.parts; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float4 o = reinterpret_cast<const float4*>(p.part_o + ((int64_t(g) * p.parts + k) * 256 + r) * 128)[lane];
+      acc.x = fmaf(wk, o.x, acc.x);
+      acc.y = fmaf(wk, o.y, acc.y);
+      acc.z = fmaf(wk, o.z, acc.z);
+      acc.w = fmaf(wk, o.w, acc.w);
+    }
+    const float inv = 1.0f / wsum;
+    const int64_t tok = int64_t(i) * p.C + pair * 256 + r;
+    uint2 packed;
+    packed.x = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.x * inv))) |
+               (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y * inv))) << 16);
+    packed.y = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.z * inv))) |
+               (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w * inv))) << 16);
+    reinterpret_cast<uint2*>(p.out + (tok * p.H + h) * 128)[lane] = packed;
+    if (lane == 0 && p.lse) p.lse[int64_t(h) * p.rc + tok] = mx + logf(wsum);
+  }
+}
+
+// Parts per unit of a plan (1: nothing to combine).
+int32_t key_parts(const wf_plan_hdr* h, const void* host_plan) {
+  if (h->num_units == 0) return 1;
+  const wf_plan_unit* u =
+      reinterpret_cast<const wf_plan_unit*>(static_cast<const uint8_t*>(host_plan) + h->off_units);
+  return u[0].parts;
+}
+
+wf_status launch_combine(const wf_plan_hdr* h, const void* host_plan, void* workspace, void* out, float* lse,
+                         cudaStream_t stream) {
+  const int32_t parts = key_parts(h, host_plan);
+  if (parts <= 1) return WF_OK;
+  CombineParams c{};
+  c.part_o = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + WF_ATTN_STATUS_BYTES);
+  c.part_lse = c.part_o + int64_t(h->num_units) * 256 * 128;
+  c.out = static_cast<__nv_bfloat16*>(out);
+  c.lse = lse;
+  c.H = h->H;
+  c.C = h->C;
+  c.q_pairs = h->q_pairs;
+  c.parts = parts;
+  c.rc = h->R * h->C;
+  const int64_t groups = int64_t(h->num_units) / parts;
+  if (groups > 0x7FFFFFFF) return WF_ERR_CAPACITY;
+  attn_combine_kernel<<<dim3(unsigned(groups), 32), 256, 0, stream>>>(c);
+  return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
 // Limit of every bounded wait in the tensor-core kernel (WF_WAIT_TIMEOUT_MS,
 // default 2000 ms), read at each launch.
 uint64_t wait_timeout_ns() {
@@ -128,7 +205,8 @@ uint64_t wait_timeout_ns() {
 extern "C" size_t wf_attn_workspace_bytes(const void* host_plan) {
   const wf_plan_hdr* h = static_cast<const wf_plan_hdr*>(host_plan);
   if (!h || h->magic != WF_PLAN_MAGIC || h->version != WF_PLAN_VERSION) return 0;
-  return WF_ATTN_STATUS_BYTES;
+  if (key_parts(h, host_plan) <= 1) return WF_ATTN_STATUS_BYTES;
+  return WF_ATTN_STATUS_BYTES + size_t(h->num_units) * 256 * (128 + 1) * sizeof(float);
 }
 
 extern "C" wf_status wf_attn_workspace_init(void* workspace, size_t workspace_bytes, wf_stream_t stream) {
@@ -163,7 +241,7 @@ extern "C" wf_status wf_chunk_causal_attn(const void* host_plan, const void* dev
   if (misaligned(dev_plan) || misaligned(q_rot) || misaligned(k_pool) || misaligned(v_pool) || misaligned(out) ||
       misaligned(workspace) || (reinterpret_cast<uintptr_t>(lse) % 4))
     return WF_ERR_ALIGNMENT;
-  if (workspace_bytes < WF_ATTN_STATUS_BYTES) return WF_ERR_WORKSPACE;
+  if (workspace_bytes < wf_attn_workspace_bytes(host_plan)) return WF_ERR_WORKSPACE;
   if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return WF_ERR_INVALID_ARG;
   const float scale = softmax_scale == 0.f ? float(1.0 / std::sqrt(double(h->D))) : softmax_scale;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -171,7 +249,9 @@ extern "C" wf_status wf_chunk_causal_attn(const void* host_plan, const void* dev
 
   if (h->dtype == WF_BF16) {
     if (h->D != 128) return WF_ERR_UNSUPPORTED;
-    return wf::launch_attn_sm100(h, dp, q_rot, k_pool, v_pool, out, lse, scale, workspace, wait_timeout_ns(), s);
+    const wf_status st =
+        wf::launch_attn_sm100(h, dp, q_rot, k_pool, v_pool, out, lse, scale, workspace, wait_timeout_ns(), s);
+    return st == WF_OK ? launch_combine(h, host_plan, workspace, out, lse, s) : st;
   }
   if (h->dtype != WF_F32 || (h->D != 64 && h->D != 128)) return WF_ERR_UNSUPPORTED;
   F32Params p{};
@@ -213,10 +293,12 @@ extern "C" wf_status wf_chunk_causal_attn_fp8(const void* host_plan, const void*
       misaligned(workspace) || (reinterpret_cast<uintptr_t>(lse) % 4) ||
       (reinterpret_cast<uintptr_t>(q_scales) % 4) || (reinterpret_cast<uintptr_t>(k_scales) % 4))
     return WF_ERR_ALIGNMENT;
-  if (workspace_bytes < WF_ATTN_STATUS_BYTES) return WF_ERR_WORKSPACE;
+  if (workspace_bytes < wf_attn_workspace_bytes(host_plan)) return WF_ERR_WORKSPACE;
   if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return WF_ERR_INVALID_ARG;
   if (h->dtype != WF_BF16 || h->D != 128) return WF_ERR_UNSUPPORTED;
   const float scale = softmax_scale == 0.f ? float(1.0 / std::sqrt(double(h->D))) : softmax_scale;
-  return wf::launch_attn_sm100_fp8(h, static_cast<const uint8_t*>(dev_plan), q8, q_scales, k8_pool, k_scales, v_pool,
-                                   out, lse, scale, workspace, wait_timeout_ns(), reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const wf_status st = wf::launch_attn_sm100_fp8(h, static_cast<const uint8_t*>(dev_plan), q8, q_scales, k8_pool,
+                                                 k_scales, v_pool, out, lse, scale, workspace, wait_timeout_ns(), s);
+  return st == WF_OK ? launch_combine(h, host_plan, workspace, out, lse, s) : st;
 }

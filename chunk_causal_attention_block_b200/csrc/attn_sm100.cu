@@ -91,6 +91,9 @@ struct Params {
   const float* q_scales;     // [R, nblk, H]
   const float* k_scales;     // [S, nblk, H]
   int32_t S, nblk;           // pool slots; scale blocks (= key tiles) per chunk
+  // split units: normalised partial O [slot][256][128] and LSE [slot][256]
+  float* part_o;
+  float* part_lse;
 };
 
 // Barrier indices in the barrier block.
@@ -182,6 +185,12 @@ __device__ __forceinline__ int first_visible_slot(const Params& p, const wf_plan
   return int((n - nvis + 1) % p.S);
 }
 
+// Key tiles [t0, t1) of a unit: its part of the chunk's n tiles.
+__device__ __forceinline__ void unit_tile_range(const wf_plan_unit& unit, int n, int& t0, int& t1) {
+  t0 = unit.part * n / unit.parts;
+  t1 = (unit.part + 1) * n / unit.parts;
+}
+
 template <bool kFp8>
 __device__ __forceinline__ int unit_key_tiles(const Params& p, const wf_plan_chunk* rec) {
   if constexpr (kFp8)
@@ -232,8 +241,9 @@ __device__ __forceinline__ void producer(const Shared& sh, const Params& p, cons
     }
     ++q_it;
     const int first_slot = kFp8 ? first_visible_slot(p, p.chunks + unit.chunk) : 0;
-    const int n_tiles = unit_key_tiles<kFp8>(p, p.chunks + unit.chunk);
-    for (int j = 0; j < n_tiles; ++j) {
+    int t0, t1;
+    unit_tile_range(unit, unit_key_tiles<kFp8>(p, p.chunks + unit.chunk), t0, t1);
+    for (int j = t0; j < t1; ++j) {
       int32_t tok, valid;
       if constexpr (kFp8) {
         int32_t slot, blk;
@@ -351,7 +361,9 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
   const uint64_t qd0 = kmajor_desc(q_tile(sh, 0)), qd1 = kmajor_desc(q_tile(sh, 1));
   for (int u = u0; u < u1 && ok; ++u) {
     const wf_plan_unit unit = p.units[u];
-    const int n = unit_key_tiles<kFp8>(p, p.chunks + unit.chunk);
+    int t0, t1;
+    unit_tile_range(unit, unit_key_tiles<kFp8>(p, p.chunks + unit.chunk), t0, t1);
+    const int n = t1 - t0;  // key tiles of this unit
     const bool live1 = p.C - unit.pair * 256 > 128;
     if (!wait_bar(sh, p, kBarQFull, q_it & 1, 10)) { ok = false; break; }
     ++q_it;
@@ -437,10 +449,11 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
       first_slot = first_visible_slot(p, p.chunks + unit.chunk);
       sl2_unit *= __ldg(p.q_scales + (int64_t(unit.chunk) * p.nblk + 2 * unit.pair + t) * p.H + unit.head);
     }
-    const int n_tiles = unit_key_tiles<kFp8>(p, p.chunks + unit.chunk);
+    int t0, t1;
+    unit_tile_range(unit, unit_key_tiles<kFp8>(p, p.chunks + unit.chunk), t0, t1);
     float m_ref = -INFINITY;  // reference max (log2 units)
     float l = 0.f;
-    for (int j = 0; j < n_tiles; ++j) {
+    for (int j = t0; j < t1; ++j) {
       int32_t tok, valid;
       float sl2 = sl2_unit;
       if constexpr (kFp8) {
@@ -477,7 +490,7 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
       }
       const float mx = fmaxf(max3f(mxs[0], mxs[1], mxs[2]), max3f(mxs[3], max3f(mxs[4], mxs[5], mxs[6]), mxs[7]));
       const float m_new = fmaxf(m_ref, mx * sl2);
-      if (j == 0) {
+      if (j == t0) {
         m_ref = m_new;
       } else {
         const bool need = m_new > m_ref + kRescaleThreshold;
@@ -525,13 +538,33 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
       tc_fence_before();
       mbar_arrive(smem_u32(sh.bars + kBarPFull + t));
     }
-    // epilogue: O / l -> bf16 rows of this tile
+    // epilogue: O / l -> bf16 rows of this tile (a part of a split unit:
+    // fp32 rows and the LSE into its partial slot, merged by the combine pass)
     if (!wait_bar(sh, p, kBarOFull + t, o_cnt & 1, 24 + t)) return;
     ++o_cnt;
     tc_fence_after();
     const float inv_l = 1.0f / l;
     const int32_t qtok = unit.chunk * p.C + unit.pair * 256 + 128 * t + row_in_tile;
     const bool store = row_in_tile < rows_here;
+    const float lse_row = (m_ref + __log2f(l)) * 0.69314718055994531f;
+    if (unit.parts > 1) {
+      const int64_t prow = int64_t(unit.slot) * 256 + 128 * t + row_in_tile;
+      float4* pdst = reinterpret_cast<float4*>(p.part_o + prow * 128);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(o_tm + 32 * q4, r);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            pdst[8 * q4 + v] = make_float4(__uint_as_float(r[4 * v]) * inv_l, __uint_as_float(r[4 * v + 1]) * inv_l,
+                                           __uint_as_float(r[4 * v + 2]) * inv_l, __uint_as_float(r[4 * v + 3]) * inv_l);
+        }
+      }
+      if (store) p.part_lse[prow] = lse_row;
+      continue;
+    }
     uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t(qtok) * p.H + unit.head) * 128);
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
@@ -550,7 +583,7 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
         }
       }
     }
-    if (store && p.lse) p.lse[int64_t(unit.head) * p.rc + qtok] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+    if (store && p.lse) p.lse[int64_t(unit.head) * p.rc + qtok] = lse_row;
   }
 }
 
@@ -692,6 +725,9 @@ wf_status launch(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q, c
   p.k_scales = k_scales;
   p.S = h->S;
   p.nblk = (h->C + 127) / 128;
+  // partial slots after the status block (used only by split units)
+  p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + WF_ATTN_STATUS_BYTES);
+  p.part_lse = p.part_o + int64_t(h->num_units) * 256 * 128;
   attn_fwd_sm100<kFp8><<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

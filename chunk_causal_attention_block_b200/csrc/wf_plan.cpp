@@ -25,7 +25,7 @@ struct Geometry {
   int32_t H, D, fh, fw, F, C, Wc, wc_eff, R, S, dtype, Pt, Ph, Pw, G;
   int64_t n0, first;
   double theta;
-  int32_t q_pairs, q_tiles;
+  int32_t q_pairs, q_tiles, parts;
   int64_t num_units;
   uint64_t off_chunks, off_vis, off_rope_t, off_rope_h, off_rope_w, off_units, off_cta, total;
 };
@@ -90,7 +90,35 @@ wf_status geometry(const wf_round_desc* d, Geometry* g, bool query_device) {
   g->first = d->n0 - g->wc_eff;
   g->q_pairs = int32_t(ceil_div(C, WF_Q_PAIR));
   g->q_tiles = int32_t(ceil_div(C, WF_Q_TILE));
-  g->num_units = int64_t(g->R) * g->H * g->q_pairs;
+  // Key split: when the round has fewer than two units per bin (a single
+  // chunk), each unit's key tiles are shared out over `parts` units, the
+  // count whose bin filling ceil(U*p/G) / (U*p/G) plus 1% per extra part is
+  // smallest (ties: fewer parts), with at least WF_MIN_PART_TILES tiles per
+  // part in the round's smallest chunk.  bf16 plans only.  With two or more
+  // units per bin the longest-first assignment and its refinement balance
+  // the bins without it.
+  const int64_t pairs_all = int64_t(g->R) * g->H * g->q_pairs;
+  {
+    const int64_t nvis0 = g->wc_eff + 1;  // chunk 0 sees the fewest keys
+    const int64_t s0 = g->first % S, len0 = std::min<int64_t>(nvis0, S - s0);
+    const int64_t tiles0 = ceil_div(len0 * C, WF_KEY_TILE) + ceil_div((nvis0 - len0) * C, WF_KEY_TILE);
+    int32_t best_p = 1;
+    int64_t best_a = 0;
+    for (int32_t p = 1; p <= WF_MAX_KEY_PARTS; ++p) {
+      if (p > 1 && (d->dtype != WF_BF16 || pairs_all >= 2 * int64_t(G) ||
+                    tiles0 < int64_t(WF_MIN_PART_TILES) * p))
+        break;
+      // score(p) = A_p / (100 U p) with A_p = 100 ceil(U p / G) G + (p - 1) U p
+      const int64_t up = pairs_all * p;
+      const int64_t a = 100 * ceil_div(up, G) * G + int64_t(p - 1) * up;
+      if (p == 1 || a * best_p < best_a * p) {
+        best_p = p;
+        best_a = a;
+      }
+    }
+    g->parts = best_p;
+  }
+  g->num_units = pairs_all * g->parts;
   if (g->num_units > (int64_t(1) << 26)) return WF_ERR_CAPACITY;
 
   uint64_t off = sizeof(wf_plan_hdr);
@@ -203,13 +231,19 @@ extern "C" wf_status wf_plan_round(const wf_round_desc* desc, void* host_plan, s
           // a second live query tile only lengthens by about a tenth (its
           // softmax overlaps the first tile's MMAs): weight 11 for two live
           // tiles, 10 for one.
-          units.push_back({i, hh, p, ch[i].key_tiles * (9 + live)});
+          const int32_t n = ch[i].key_tiles, P = g.parts;
+          for (int32_t k = 0; k < P; ++k) {
+            const int32_t tiles = (k + 1) * n / P - k * n / P;
+            const int32_t slot = P > 1 ? ((i * g.H + hh) * g.q_pairs + p) * P + k : -1;
+            units.push_back({i, hh, p, tiles * (9 + live), k, P, slot, 0});
+          }
         }
     std::sort(units.begin(), units.end(), [](const wf_plan_unit& a, const wf_plan_unit& b) {
       if (a.cost != b.cost) return a.cost > b.cost;
       if (a.chunk != b.chunk) return a.chunk > b.chunk;
       if (a.head != b.head) return a.head < b.head;
-      return a.pair < b.pair;
+      if (a.pair != b.pair) return a.pair < b.pair;
+      return a.part < b.part;
     });
     // Greedy start: each unit, longest first, to the least-loaded bin
     // (lowest index on ties).

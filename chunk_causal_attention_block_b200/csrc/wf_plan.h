@@ -7,7 +7,7 @@
 #include <stdint.h>
 
 #define WF_PLAN_MAGIC 0x31504657u  // "WFP1" little-endian
-#define WF_PLAN_VERSION 1u
+#define WF_PLAN_VERSION 2u
 #define WF_KEY_TILE 128            // keys per attention tile
 #define WF_Q_TILE 128              // query rows per tensor-core tile
 #define WF_Q_PAIR 256              // query rows per attention work unit (two tiles)
@@ -30,11 +30,21 @@ struct wf_plan_chunk {
 static_assert(sizeof(wf_plan_chunk) == 56, "chunk record layout");
 
 // One attention work unit: query rows [pair*256, min(C, pair*256+256)) of
-// in-round chunk `chunk`, head `head`; cost = key_tiles * (9 + live 128-row
-// tiles): a unit's time is dominated by its per-key-tile pipeline latency.
+// in-round chunk `chunk`, head `head`, against part `part` of `parts` equal
+// shares of the chunk's key tiles (tiles [part*n/parts, (part+1)*n/parts),
+// n the kernel's tile count; parts = 1: all of them).  A split unit writes
+// its normalised partial O and LSE to partial slot `slot` of the attention
+// workspace and a combine pass merges the parts (slot = -1 when parts = 1).
+// cost = its key tiles * (9 + live 128-row tiles): a unit's time is
+// dominated by its per-key-tile pipeline latency.
 struct wf_plan_unit {
   int32_t chunk, head, pair, cost;
+  int32_t part, parts, slot, pad;
 };
+static_assert(sizeof(wf_plan_unit) == 32, "unit record layout");
+
+#define WF_MAX_KEY_PARTS 8        // most parts a unit's keys are split into
+#define WF_MIN_PART_TILES 8       // fewest 128-key tiles a part may hold
 
 struct wf_plan_hdr {
   uint32_t magic;        // 0
@@ -61,6 +71,8 @@ static_assert(offsetof(wf_plan_hdr, n0) == 96, "header layout");
 static_assert(offsetof(wf_plan_hdr, off_chunks) == 120, "header layout");
 
 #define WF_ATTN_STATUS_BYTES 256  // status word block at the start of the workspace
+// After it, for plans with split units: partial O [slots][256 rows][128] fp32,
+// then partial LSE [slots][256 rows] fp32 (slots = number of units).
 
 // Device-side status record at the start of an attention workspace.
 struct wf_dev_status {

@@ -160,6 +160,15 @@ class Rollout:
         wf.wf_plan_round(d, buf, self.dev_plan, self.stream, host_bytes=buf.numel(), dev_bytes=self.dev_plan.numel())
         self._plan_events[k].record(self.stream)
         self.host_plan = buf
+        self._ensure_workspace(wf.wf_attn_workspace_bytes(buf))
+
+    def _ensure_workspace(self, n: int):
+        """The attention workspace: a status block, plus partial slots when the plan splits units' keys."""
+        if n <= self.workspace.numel():
+            return
+        self.stream.synchronize()
+        self.workspace = torch.empty(n, dtype=torch.uint8, device=self.device)
+        wf.wf_attn_workspace_init(self.workspace, self.stream, nbytes=wf.WF_ATTN_STATUS_BYTES)
 
     # ------------------------------------------------------------- inputs
     def fill_inputs(self, n_first: int, nchunks: int, tag: int):

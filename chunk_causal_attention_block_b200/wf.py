@@ -25,6 +25,7 @@ WF_F32, WF_BF16 = 0, 1
 WF_MAX_INROUND = 16
 WF_SYNTH_Q, WF_SYNTH_K, WF_SYNTH_V = 1, 2, 3
 WF_FP8_BLOCK = 128
+WF_ATTN_STATUS_BYTES = 256
 WF_FP8_Q, WF_FP8_K = 0, 1
 
 # exported symbols, in the order include/wf.h and include/wf_synth.h declare them
@@ -245,9 +246,11 @@ def decode_plan(blob) -> dict:
     h["rope_h"] = table(h["off_rope_h"], h["fh"], h["Ph"])
     h["rope_w"] = table(h["off_rope_w"], h["fw"], h["Pw"])
     cta = np.frombuffer(b, dtype=np.int32, count=h["num_ctas"] + 1, offset=h["off_cta"])
-    units = np.frombuffer(b, dtype=np.int32, count=4 * h["num_units"], offset=h["off_units"]).reshape(-1, 4)
-    h["per_cta"] = [[tuple(int(x) for x in units[u]) for u in range(cta[c], cta[c + 1])]
+    units = np.frombuffer(b, dtype=np.int32, count=8 * h["num_units"], offset=h["off_units"]).reshape(-1, 8)
+    # (chunk, head, pair, cost, part, parts, slot) per unit
+    h["per_cta"] = [[tuple(int(x) for x in units[u][:7]) for u in range(cta[c], cta[c + 1])]
                     for c in range(h["num_ctas"])]
+    h["key_parts"] = int(units[0][5]) if h["num_units"] else 1
     return h
 
 

@@ -109,7 +109,10 @@ size_t wf_plan_bytes(const wf_round_desc* desc);
  * the plan lists with their 128-key tile counts.  It also holds the fp64
  * cos/sin tables of the round's RoPE angles and the attention work list:
  * units of (chunk, head, 256 query rows) in longest-first order, assigned
- * greedily to `num_ctas` bins.
+ * greedily to `num_ctas` bins and then rebalanced by moves and swaps.  When a
+ * bf16 round has fewer than two units per bin (a single chunk), every unit's
+ * key tiles are shared out over up to 8 parts (the count that fills the bins
+ * best, each part at least 8 tiles); the attention then merges the parts.
  *
  * host_plan: host buffer of >= wf_plan_bytes(desc) bytes, filled on return.
  * dev_plan:  device buffer of the same size, or NULL.  If non-NULL the blob
@@ -147,7 +150,9 @@ wf_status wf_rope3d_append(const void* host_plan, const void* dev_plan,
                            const void* q, const void* k, const void* v,
                            void* q_rot, void* k_pool, void* v_pool, wf_stream_t stream);
 
-/* Bytes of attention workspace the plan's kernels need (>= 256). */
+/* Bytes of attention workspace the plan's kernels need: the 256-byte status
+ * block, plus 256 rows x (128 + 1) fp32 per unit when the plan splits units'
+ * keys (see wf_plan_round); 0 for an invalid plan. */
 size_t wf_attn_workspace_bytes(const void* host_plan);
 
 /*
@@ -183,7 +188,9 @@ wf_status wf_attn_workspace_status(const void* workspace, wf_stream_t stream, in
  * softmax_scale: 0 means 1/sqrt(D).
  * workspace: device buffer of >= wf_attn_workspace_bytes(host_plan) bytes,
  *            zeroed once by wf_attn_workspace_init.  Calls that overlap on
- *            the GPU may share one workspace.
+ *            the GPU may share one workspace unless the plan splits units'
+ *            keys: their partial rows live there until the combine pass (a
+ *            second kernel on `stream`) has merged them.
  * Errors: WF_ERR_PLAN, WF_ERR_INVALID_ARG, WF_ERR_ALIGNMENT,
  *         WF_ERR_UNSUPPORTED, WF_ERR_WORKSPACE, WF_ERR_CUDA.
  */

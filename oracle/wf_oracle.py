@@ -38,6 +38,7 @@ Readings where the pages are silent (each is a parameter or a stated choice):
 from __future__ import annotations
 
 import math
+from fractions import Fraction
 
 import numpy as np
 
@@ -155,8 +156,31 @@ def ring_contents_after(appends, S: int):
 # plan re-derivation (visibility, slots, segments, work list)
 # --------------------------------------------------------------------------
 
-def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas):
-    """Re-derive the round plan: per-chunk visibility/slots and the LPT work list."""
+MAX_KEY_PARTS = 8     # most parts a unit's key tiles are shared over
+MIN_PART_TILES = 8    # fewest key tiles per part in the round's smallest chunk
+
+
+def key_parts(units_unsplit: int, num_ctas: int, tiles_min: int, split: bool) -> int:
+    """Number of parts each unit's key tiles are shared over.  1 without
+    `split` (fp32 plans) or with two or more units per bin; otherwise the p
+    (at most MAX_KEY_PARTS, each part at least MIN_PART_TILES tiles of the
+    smallest chunk) minimising the bin filling ceil(U*p/G) / (U*p/G) plus 1%
+    per extra part; ties to fewer parts."""
+    best_p, best = 1, None
+    for p in range(1, MAX_KEY_PARTS + 1):
+        if p > 1 and (not split or units_unsplit >= 2 * num_ctas or tiles_min < MIN_PART_TILES * p):
+            break
+        up = units_unsplit * p
+        score = Fraction(-(-up // num_ctas) * num_ctas, up) + Fraction(p - 1, 100)
+        if best is None or score < best:
+            best_p, best = p, score
+    return best_p
+
+
+def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas, split=None):
+    """Re-derive the round plan: per-chunk visibility/slots and the LPT work list.
+    split: share units' keys over several parts when units are few (default:
+    for the 16-bit path, D = 128)."""
     C = F * fh * fw
     wc_eff = min(Wc, n0)
     first = n0 - wc_eff
@@ -173,14 +197,20 @@ def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas):
                            vis_chunks=vis, vis_slots=[v % S for v in vis],
                            keys=nvis * C, segs=segs, key_tiles=tiles))
     pairs = -(-C // Q_PAIR)
+    split = (D == 128) if split is None else split
+    P = key_parts(R * H * pairs, num_ctas, chunks[0]["key_tiles"], split)
     units = []
     for i in range(R):
         for h in range(H):
             for p in range(pairs):
                 rows = min(Q_PAIR, C - Q_PAIR * p)
                 live = 1 if rows <= Q_TILE else 2
-                units.append((i, h, p, chunks[i]["key_tiles"] * (9 + live)))
-    units.sort(key=lambda u: (-u[3], -u[0], u[1], u[2]))
+                n = chunks[i]["key_tiles"]
+                for k in range(P):
+                    tiles = (k + 1) * n // P - k * n // P
+                    slot = ((i * H + h) * pairs + p) * P + k if P > 1 else -1
+                    units.append((i, h, p, tiles * (9 + live), k, P, slot))
+    units.sort(key=lambda u: (-u[3], -u[0], u[1], u[2], u[4]))
     loads = [0] * num_ctas
     per_cta = [[] for _ in range(num_ctas)]
     for u in units:
@@ -224,7 +254,7 @@ def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas):
         per_cta[b].append(x)
         loads[b] += x[3]
     return dict(C=C, wc_eff=wc_eff, first=first, chunks=chunks, units=units,
-                per_cta=per_cta, loads=loads, q_pairs=pairs)
+                per_cta=per_cta, loads=loads, q_pairs=pairs, key_parts=P)
 
 
 # --------------------------------------------------------------------------

@@ -143,9 +143,27 @@ def test_fp8_entry_points_reject_bad_arguments_before_any_launch():
         assert e.value.code == code
 
 
+def test_workspace_size_follows_the_key_split():
+    # one 1560-token chunk, 2 heads: 14 units for 148 CTAs -> each unit's keys in 4 parts
+    d = wf.make_desc(2, 128, 30, 52, 1, 2, 1, 2, [1000], dtype=wf.WF_BF16, num_ctas=148)
+    host = _plan(d)
+    p = wf.decode_plan(host)
+    assert p["key_parts"] == 4 and p["num_units"] == 56
+    assert wf.wf_attn_workspace_bytes(host) == 256 + 56 * 256 * 129 * 4
+    fake = 1 << 20
+    with pytest.raises(wf.WfError) as e:  # too small for the partial slots: rejected before any launch
+        wf.wf_chunk_causal_attn(host, fake, fake, fake, fake, fake, None, 0.0, fake, workspace_bytes=4096)
+    assert e.value.code == wf.WF_ERR_WORKSPACE
+    with pytest.raises(wf.WfError) as e:  # more than the static scratch of the allocation-free entry point
+        wf.wf_chunk_causal_attn_noalloc(host, fake, fake, fake, fake, fake, None, 0.0)
+    assert e.value.code == wf.WF_ERR_CAPACITY
+    # an unsplit plan needs the status block only
+    assert wf.wf_attn_workspace_bytes(_plan(_desc())) == 256
+
+
 def _compare_plan(host, ref, desc_kw):
     p = wf.decode_plan(host)
-    assert p["magic"] == 0x31504657 and p["version"] == 1
+    assert p["magic"] == 0x31504657 and p["version"] == 2
     assert p["C"] == ref["C"] and p["wc_eff"] == ref["wc_eff"] and p["first"] == ref["first"]
     for got, want in zip(p["chunks"], ref["chunks"]):
         for key in ("n", "slot", "noise", "nvis", "keys", "key_tiles", "vis_slots"):
@@ -182,7 +200,7 @@ def test_plan_matches_oracle_rederivation(case):
                      S=kw["S"], dtype=dtype, num_ctas=kw["num_ctas"])
     host = _plan(d)
     ref = orc.plan_round(kw["H"], kw["D"], kw["fh"], kw["fw"], kw["F"], kw["Wc"], kw["R"], kw["S"], kw["n0"],
-                         kw["noise_t"], kw["num_ctas"])
+                         kw["noise_t"], kw["num_ctas"], split=dtype == wf.WF_BF16)
     _compare_plan(host, ref, kw)
 
 

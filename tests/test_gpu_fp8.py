@@ -58,6 +58,7 @@ SMALL = [
     RoundConfig("tiny chunks", H=3, D=128, fh=5, fw=7, F=2, Wc=2, R=4, noise_t=(0, 250, 500, 750)),
     RoundConfig("C=1", H=2, D=128, fh=1, fw=1, F=1, Wc=5, R=4, noise_t=(250, 500, 750, 1000)),
     RoundConfig("no cache", H=2, D=128, fh=9, fw=13, F=2, Wc=0, R=1, noise_t=(1000,)),
+    RoundConfig("key split", H=2, D=128, fh=30, fw=52, F=1, Wc=2, R=1, noise_t=(1000,)),
 ]
 
 
@@ -73,7 +74,8 @@ def test_fp8_codes_bit_exact_and_attention_all_rows(cfg):
     gc.run_rollout(cfg, (0, 1, cfg.Wc + cfg.R + 1), on_round=on_round, fp8=True)
 
 
-@pytest.mark.parametrize("name,heads,rounds", [("wan13b_round", [2, 9], (0, 7)), ("wan14b_round", [5, 33], (0,))])
+@pytest.mark.parametrize("name,heads,rounds", [("wan13b_round", [2, 9], (0, 7)), ("wan14b_round", [5, 33], (0,)),
+                                               ("wan13b_single", [3], (0,))])
 def test_fp8_full_size_sampled(name, heads, rounds):
     cfg = CONFIGS[name]
     rows = gc.sample_rows(cfg, extra=12)

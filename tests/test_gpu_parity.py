@@ -92,6 +92,8 @@ SMALL_BF16 = [
     RoundConfig("C=1", H=2, D=128, fh=1, fw=1, F=1, Wc=5, R=4, noise_t=(250, 500, 750, 1000)),
     # the most in-round chunks a round may hold (16), ragged 42-token chunks
     RoundConfig("R=16", H=1, D=128, fh=6, fw=7, F=1, Wc=3, R=16, noise_t=tuple(60 * i for i in range(16))),
+    # 14 units for 148 CTAs: every unit's keys split in 4 parts, merged by the combine pass
+    RoundConfig("key split", H=2, D=128, fh=30, fw=52, F=1, Wc=2, R=1, noise_t=(1000,)),
 ]
 
 

@@ -210,16 +210,56 @@ def test_plan_tile_pairs_match_brute_mask():
             assert ch["key_tiles"] == sum(-(-ln // 128) for _, ln in ch["segs"] if ln)
 
 
-def test_plan_work_list_covers_every_row_once():
-    p = orc.plan_round(3, 128, 30, 52, 3, 7, 4, 11, 7, [250, 500, 750, 1000], 148)
-    rows = set()
+def _covered_row_tiles(p):
+    """Check that the units cover every (chunk, head, query row, key tile) exactly once:
+    each row pair's parts partition [0, key_tiles).  Returns the number covered."""
+    ranges = {}
     for lst in p["per_cta"]:
-        for (i, h, pp, cost) in lst:
-            for r in range(pp * 256, min(p["C"], pp * 256 + 256)):
-                assert (i, h, r) not in rows
-                rows.add((i, h, r))
-    assert len(rows) == 4 * 3 * p["C"]
+        for (i, h, pp, cost, k, P, slot) in lst:
+            n = p["chunks"][i]["key_tiles"]
+            t0, t1 = k * n // P, (k + 1) * n // P
+            rows = min(256, p["C"] - pp * 256)
+            assert rows > 0
+            assert cost == (t1 - t0) * (9 + (1 if rows <= 128 else 2))
+            ranges.setdefault((i, h, pp), []).append((t0, t1, rows))
+    total = 0
+    for (i, h, pp), rs in ranges.items():
+        rs.sort()
+        n = p["chunks"][i]["key_tiles"]
+        assert rs[0][0] == 0 and rs[-1][1] == n
+        assert all(a[1] == b[0] for a, b in zip(rs, rs[1:]))      # contiguous, no overlap
+        total += rs[0][2] * n
+    pairs = -(-p["C"] // 256)
+    heads = len({h for (_, h, _) in ranges})
+    assert len(ranges) == len(p["chunks"]) * heads * pairs                 # every (chunk, head, pair)
+    return total
+
+
+def test_plan_work_list_covers_every_row_once():
+    # 12 heads: 912 units on 148 bins, no key split
+    p = orc.plan_round(12, 128, 30, 52, 3, 7, 4, 11, 7, [250, 500, 750, 1000], 148)
+    assert p["key_parts"] == 1
+    assert _covered_row_tiles(p) == sum(p["C"] * 12 * ch["key_tiles"] for ch in p["chunks"])
     assert max(p["loads"]) - min(p["loads"]) <= max(u[3] for u in p["units"])
+    # 3 heads: 228 units (< 2 per bin), split in 5 (see the single-chunk case below)
+    p = orc.plan_round(3, 128, 30, 52, 3, 7, 4, 11, 7, [250, 500, 750, 1000], 148)
+    assert p["key_parts"] == 5
+    assert _covered_row_tiles(p) == sum(p["C"] * 3 * ch["key_tiles"] for ch in p["chunks"])
+    assert max(p["loads"]) - min(p["loads"]) <= max(u[3] for u in p["units"])
+
+
+def test_plan_key_split_of_a_single_chunk():
+    # 12 heads x 19 row pairs of one 4680-token chunk = 228 units on 148 bins.  Bin filling
+    # ceil(228p/148) / (228p/148) + (p-1)/100 for p = 1..8: 1.298, 1.308, 1.102, 1.166, 1.079,
+    # 1.132, 1.080, 1.125 -> p = 5 (fewest tiles per part 256/5 >= 8).
+    p = orc.plan_round(12, 128, 30, 52, 3, 6, 1, 7, 6, [1000], 148)
+    assert p["key_parts"] == 5
+    n = p["chunks"][0]["key_tiles"]
+    assert n == 256 and _covered_row_tiles(p) == 12 * 4680 * n
+    slots = sorted(u[6] for lst in p["per_cta"] for u in lst)
+    assert slots == list(range(228 * 5))
+    # the 16-bit-only rule: no split for fp32 plans
+    assert orc.plan_round(12, 128, 30, 52, 3, 6, 1, 7, 6, [1000], 148, split=False)["key_parts"] == 1
 
 
 # ---------------------------------------------------------------- mask / attention
