@@ -132,3 +132,15 @@ def test_fp8_stream_start_and_refresh_round():
     ref_cfg = CONFIGS["wan13b_refresh"]
     srows = gc.sample_rows(ref_cfg, extra=8)
     gc.run_rollout(ref_cfg, (0,), on_round=lambda ro, r: gc.check_attention(ro, r, [6], srows, "refresh"), fp8=True)
+
+
+def test_fp8_720p_long_rollout_sampled():
+    # the largest shape over 200 rounds: codes bit-exact and attention within the gates at the checked rounds
+    cfg = CONFIGS["p720_rollout"]
+    rows = gc.sample_rows(cfg, extra=4)
+
+    def on_round(ro, r):
+        _check_codes(ro, r, [29])
+        gc.check_attention(ro, r, [29], rows, f"720p fp8 r{r}")
+
+    gc.run_rollout(cfg, cfg.check_rounds, on_round=on_round, fp8=True)
