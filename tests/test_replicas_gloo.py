@@ -2,7 +2,9 @@
 
 The wave-round path has no exchange step, so N GPUs run N independent
 replicas; the only collectives are the barrier and the max over ranks of the
-device time.  These run here on the gloo backend with world size 2.
+device time.  These run here on the gloo backend with world size 2, including
+a replica that leaves between steps: the surviving rank's reduction ends with
+an error within the process group's timeout instead of waiting for good.
 """
 import importlib.util
 import os
@@ -64,3 +66,38 @@ def test_single_rank_needs_no_process_group():
     bench = _load_bench()
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.replica_seed(0) == 42
+
+
+def _worker_rank_dies(rank, world, port, out):
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        # a replica that fails between steps: it leaves without joining the timing reduction
+        dist.destroy_process_group()
+        out[rank] = "left"
+        return
+    bench = _load_bench()
+    t0 = time.time()
+    try:
+        bench.max_over_ranks(10.0, world)
+        out[rank] = ("no error", time.time() - t0)
+    except Exception as e:  # the surviving rank learns of the failure instead of waiting for good
+        out[rank] = (type(e).__name__, time.time() - t0)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+def test_a_replica_that_leaves_ends_the_others_reduction_with_an_error():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker_rank_dies, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[1] == "left"
+    kind, waited = res[0]
+    assert kind != "no error" and waited < 60, res
