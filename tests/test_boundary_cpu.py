@@ -239,3 +239,24 @@ def test_plan_rope_tables_match_oracle_angles(D, pairs):
         tol = 4e-16 * np.maximum(1, np.abs(ang))
         assert np.all(np.abs(got_c - np.cos(ang)) <= tol)
         assert np.all(np.abs(got_s - np.sin(ang)) <= tol)
+
+
+def test_random_round_shapes_plan_bit_exact_against_the_oracle():
+    """Random shapes, positions, ring sizes and CTA counts (split and unsplit work lists)."""
+    rng = np.random.default_rng(2024)
+    for _ in range(200):  # about one in six draws splits units' keys
+        D = int(rng.choice([64, 128]))
+        dtype = wf.WF_BF16 if D == 128 else wf.WF_F32
+        R = int(rng.integers(1, 7))
+        Wc = int(rng.integers(0, 9))
+        S = Wc + R + int(rng.integers(0, 4))
+        kw = dict(H=int(rng.integers(1, 13)), D=D, fh=int(rng.integers(1, 40)), fw=int(rng.integers(1, 40)),
+                  F=int(rng.integers(1, 4)), Wc=Wc, R=R, S=S, n0=int(rng.integers(0, 300)),
+                  noise_t=sorted(int(x) for x in rng.integers(0, 1001, R)), num_ctas=int(rng.integers(1, 300)))
+        d = wf.make_desc(kw["H"], kw["D"], kw["fh"], kw["fw"], kw["F"], kw["Wc"], kw["R"], kw["n0"], kw["noise_t"],
+                         S=kw["S"], dtype=dtype, num_ctas=kw["num_ctas"])
+        host = _plan(d)
+        ref = orc.plan_round(kw["H"], kw["D"], kw["fh"], kw["fw"], kw["F"], kw["Wc"], kw["R"], kw["S"], kw["n0"],
+                             kw["noise_t"], kw["num_ctas"], split=dtype == wf.WF_BF16)
+        _compare_plan(host, ref, kw)
+        assert wf.decode_plan(host)["key_parts"] == ref["key_parts"], kw
