@@ -52,7 +52,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_reduce_max_and_split_seeds():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)
@@ -94,7 +94,7 @@ def _worker_rank_dies(rank, world, port, out):
 
 def test_a_replica_that_leaves_ends_the_others_reduction_with_an_error():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker_rank_dies, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)
