@@ -144,3 +144,36 @@ def test_fp8_720p_long_rollout_sampled():
         gc.check_attention(ro, r, [29], rows, f"720p fp8 r{r}")
 
     gc.run_rollout(cfg, cfg.check_rounds, on_round=on_round, fp8=True)
+
+
+def test_negative_controls_fail_the_gates():
+    """Mistakes planted in the oracle (on the CPU) must fail the gates the GPU output passes."""
+    from oracle import wf_oracle as orc
+    cfg = SMALL[-1]  # the key-split round: 4 parts per unit, merged by the combine pass
+    rows = np.arange(cfg.R * cfg.C)
+    ro = gc.run_rollout(cfg, (0,), fp8=True)
+    assert wf.decode_plan(ro.host_plan)["key_parts"] > 1
+    arrays = gc.oracle_inputs(cfg, ro.n0_of(0), ro.first_n0, [0, 1], seed=ro.seed)
+    ref = gc.oracle_call(cfg, ro.n0_of(0), arrays, rows, fp8=True)
+    got = gc.to_np(ro.out[rows][:, [0, 1]])
+    gc.assert_bf16_close(got, ref["O"], "positive")
+    H, D, C = 2, cfg.D, cfg.C
+    q = orc.fp8_dequantize(ref["q8"], ref["q_scales"], C)
+    k = orc.fp8_dequantize(ref["k8"], ref["k_scales"], C)
+    v = np.concatenate([ref["v_cache"], ref["v"]]).reshape(-1, H, D)
+    mask = orc.visibility_mask(C, min(cfg.Wc, ro.n0_of(0)), cfg.R, q_chunks=rows // C)
+
+    def attend(kk, vv, m):
+        return np.stack([orc.attention(q[rows][:, h], kk[:, h], vv[:, h], m, 1 / np.sqrt(D))[0] for h in range(H)],
+                        axis=1)
+
+    # the key scales left out (codes read as values times one common scale)
+    k_unscaled = ref["k8"] * ref["k_scales"].mean()
+    with pytest.raises(AssertionError):
+        gc.assert_bf16_close(got, attend(k_unscaled, v, mask), "key scales ignored")
+    # one of the parts dropped: only the first three quarters of the keys
+    n_keys = k.shape[0]
+    keep = np.zeros(n_keys, bool)
+    keep[: 3 * n_keys // 4] = True
+    with pytest.raises(AssertionError):
+        gc.assert_bf16_close(got, attend(k, v, mask & keep[None, :]), "a key part dropped")
