@@ -286,6 +286,15 @@ def run_wf(args, rank, world, local_rank):
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
+    # host time of planning one round (wf_plan_round without the device copy),
+    # reported beside the device-timed step
+    plan_host = torch.empty(wf.wf_plan_bytes(ro.desc(ro.n0_of(W + K))), dtype=torch.uint8)
+    plan_ts = []
+    for r in range(10):
+        t0 = time.perf_counter()
+        wf.wf_plan_round(ro.desc(ro.n0_of(W + K + r)), plan_host)
+        plan_ts.append(time.perf_counter() - t0)
+    plan_ms = 1e3 * statistics.median(plan_ts)
     ms = t_start.elapsed_time(t_end)
     rope_ms = [e[0].elapsed_time(e[1]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
@@ -410,6 +419,7 @@ def run_wf(args, rank, world, local_rank):
                           f"K/V pool {2 * cfg.slots * cfg.C * cfg.H * cfg.D * elem / 1e6:.0f} MB, "
                           "fresh inputs each step)")},
         "wave_rounds_per_s": K * world / (ms_max / 1e3),
+        "plan_ms_host": plan_ms,
         "attn_tflops_kernel": achieved,
         "pct_bf16_peak": {"of_spec_2250": 100 * achieved / 2250.0,
                           f"of_{peak_kind}_burst": 100 * achieved / peak,
