@@ -162,7 +162,7 @@ def oracle_sample(cfg, seconds: float, first_n0: int, n0: int, seed: int = 42):
     import numpy as np
     from tests import gpu_common as gc
 
-    rows_per_chunk = 256
+    rows_per_chunk = min(256, cfg.C)
     rows = np.concatenate([i * cfg.C + np.arange(rows_per_chunk) for i in range(cfg.R)])
     flops_per_head = sum(4.0 * cfg.D * rows_per_chunk * k for k in cfg.visible_keys())
     done, heads, t_total = 0.0, 0, 0.0

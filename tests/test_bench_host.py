@@ -1,0 +1,57 @@
+"""Host logic of bench.py on the CPU: the kernel-code hash that keeps a DRAM
+traffic capture attached to the code it measured, and the reference arm's
+JSON line (the CPU oracle on a bounded sample)."""
+import importlib.util
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "chunk_causal_attention_block_b200", "csrc")
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_host", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _reader(edit=None):
+    def read(name):
+        with open(os.path.join(CSRC, name)) as f:
+            text = f.read()
+        return edit(name, text) if edit else text
+    return read
+
+
+def test_kernel_hash_ignores_comments_and_blank_lines_but_not_code():
+    bench = _bench()
+    base = bench.kernel_source_sha()
+    assert bench.kernel_source_sha(_reader()) == base
+    commented = _reader(lambda n, t: t.replace("\n", "\n\n// a note\n", 3) if n == "attn_sm100.cu" else t)
+    assert bench.kernel_source_sha(commented) == base
+    changed = _reader(lambda n, t: t.replace("kStages = 4", "kStages = 5") if n == "attn_sm100.cu" else t)
+    assert bench.kernel_source_sha(changed) != base
+
+
+def test_traffic_capture_is_attached_only_to_the_code_it_measured(monkeypatch):
+    bench = _bench()
+    got = bench.dram_traffic("wan13b_round")
+    assert got is None or got > 431e6  # at least the algorithmic bytes when attached
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda read=None: "0000000000000000")
+    assert bench.dram_traffic("wan13b_round") is None
+
+
+def test_reference_arm_line_has_the_contract_fields():
+    bench = _bench()
+
+    class Args:
+        config, steps, warmup, gpus = "tiny_f32", 1, 0, 1
+
+    line = bench.run_reference(Args, 0, 1)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert bench.run_reference(Args, 1, 2) is None  # other ranks do no work
