@@ -260,3 +260,18 @@ def test_random_round_shapes_plan_bit_exact_against_the_oracle():
                              kw["noise_t"], kw["num_ctas"], split=dtype == wf.WF_BF16)
         _compare_plan(host, ref, kw)
         assert wf.decode_plan(host)["key_parts"] == ref["key_parts"], kw
+
+
+def test_planning_a_round_is_fast_enough_to_overlap_the_previous_one():
+    """Host planning must stay far below a round's device time (4 ms for the 1.3B round, 85 ms at 720p)."""
+    import time
+    cases = [(12, 30, 52, 7, 4, 148, 2.0), (40, 45, 80, 7, 4, 148, 20.0), (12, 30, 52, 6, 1, 148, 2.0)]
+    for H, fh, fw, Wc, R, ctas, limit_ms in cases:
+        d = wf.make_desc(H, 128, fh, fw, 3, Wc, R, Wc + 40, [250, 500, 750, 1000][:R] if R > 1 else [1000],
+                         dtype=wf.WF_BF16, num_ctas=ctas)
+        host = _plan(d)
+        t0 = time.perf_counter()
+        for _ in range(5):
+            wf.wf_plan_round(d, host)
+        ms = (time.perf_counter() - t0) / 5 * 1e3
+        assert ms < limit_ms, (H, fh, fw, R, ms)
