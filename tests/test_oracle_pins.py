@@ -491,3 +491,23 @@ def test_fp8_round_equals_16_bit_round_when_quantization_is_exact():
     b = orc.wave_round(q, k, v, empty, empty, fp8=True, **kw)
     assert np.array_equal(b["q8"] * 2.0 ** -8, a["q_rot"].reshape(-1, H, D))
     assert np.array_equal(a["O"], b["O"]) and np.array_equal(a["LSE"], b["LSE"])
+
+
+def test_fp8_block_quantize_matches_a_torch_pipeline():
+    # the same definition written with torch: fp32 amax, fp32 448/amax and amax/448, fp32 product,
+    # torch's float8_e4m3fn conversion (nearest-even; products stay within its range)
+    rng = np.random.default_rng(5)
+    C, H, D = 300, 3, 32
+    x = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(
+        (rng.standard_normal((2 * C, H, D)) * np.exp2(rng.integers(-3, 4, (1, H, 1)))).astype(np.float32)))
+    codes, scales = orc.fp8_block_quantize(x.astype(np.float64), C)
+    t = torch.from_numpy(x.astype(np.float32))
+    for c in range(2):
+        for b in range(-(-C // 128)):
+            lo, hi = c * C + b * 128, c * C + min(C, (b + 1) * 128)
+            blk = t[lo:hi]
+            amax = blk.abs().amax(dim=(0, 2))
+            inv = torch.tensor(448.0, dtype=torch.float32) / amax
+            q = (blk * inv[None, :, None]).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+            assert np.array_equal(codes[lo:hi], q), (c, b)
+            assert np.array_equal(scales[c, b], (amax / torch.tensor(448.0)).to(torch.float64).numpy())
