@@ -145,6 +145,79 @@ void fill_rope(double* dst, int64_t npos, const int64_t* pos, int32_t P, double 
   }
 }
 
+// Work balancer.  Longest first: items ordered by cost (largest first,
+// equal costs in their given order) each go to the least-loaded bin (lowest
+// index on ties).  Refinement: with ~6 large units per bin the greedy start
+// leaves the heaviest bin ~10% above the mean, so repeatedly move one item out
+// of the heaviest bin h (lowest index on ties), or swap it for a lighter one,
+// choosing the change that leaves the two bins' larger load smallest, from the
+// lightest bin (lowest index on ties) that offers any change lowering L_h.
+// Ties keep the first candidate in bin order, item order, move before swap;
+// arriving items go to the end of their new bin.  Right after the greedy start
+// no move can lower L_h (the last item placed in a bin is its smallest and was
+// placed when that bin was the lightest), so moves only follow swaps.
+void balance(const std::vector<int64_t>& cost, int32_t G, std::vector<std::vector<int32_t>>& bins) {
+  const int32_t n = int32_t(cost.size());
+  std::vector<int32_t> order(n);
+  for (int32_t i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return cost[a] > cost[b]; });
+  using Bin = std::pair<int64_t, int32_t>;  // (load, index): min-heap pops lowest load, then index
+  std::priority_queue<Bin, std::vector<Bin>, std::greater<Bin>> heap;
+  for (int32_t c = 0; c < G; ++c) heap.push({0, c});
+  bins.assign(size_t(G), {});
+  std::vector<int64_t> load(G, 0);
+  for (int32_t i : order) {
+    const Bin b = heap.top();
+    heap.pop();
+    bins[b.second].push_back(i);
+    load[b.second] += cost[i];
+    heap.push({load[b.second], b.second});
+  }
+  std::vector<int32_t> by_load(G);
+  for (int iter = 0; iter < 5000; ++iter) {
+    int32_t h = 0;
+    for (int32_t c = 1; c < G; ++c)
+      if (load[c] > load[h]) h = c;
+    for (int32_t c = 0; c < G; ++c) by_load[c] = c;
+    std::stable_sort(by_load.begin(), by_load.end(), [&](int32_t a, int32_t b) { return load[a] < load[b]; });
+    int64_t best = -1;
+    int32_t best_b = -1, best_x = -1, best_y = -1;
+    for (int32_t b : by_load) {
+      if (b == h) continue;
+      if (load[b] >= load[h]) break;
+      for (int32_t xi = 0; xi < int32_t(bins[h].size()); ++xi) {
+        const int64_t x = cost[bins[h][xi]];
+        const int64_t mv = std::max(load[h] - x, load[b] + x);
+        if (mv < load[h] && (best < 0 || mv < best)) {
+          best = mv; best_b = b; best_x = xi; best_y = -1;
+        }
+        for (int32_t yi = 0; yi < int32_t(bins[b].size()); ++yi) {
+          const int64_t d = x - cost[bins[b][yi]];
+          if (d <= 0) continue;
+          const int64_t sw = std::max(load[h] - d, load[b] + d);
+          if (sw < load[h] && (best < 0 || sw < best)) {
+            best = sw; best_b = b; best_x = xi; best_y = yi;
+          }
+        }
+      }
+      if (best >= 0) break;
+    }
+    if (best < 0) break;
+    const int32_t x = bins[h][best_x];
+    bins[h].erase(bins[h].begin() + best_x);
+    load[h] -= cost[x];
+    if (best_y >= 0) {
+      const int32_t y = bins[best_b][best_y];
+      bins[best_b].erase(bins[best_b].begin() + best_y);
+      load[best_b] -= cost[y];
+      bins[h].push_back(y);
+      load[h] += cost[y];
+    }
+    bins[best_b].push_back(x);
+    load[best_b] += cost[x];
+  }
+}
+
 }  // namespace
 
 extern "C" size_t wf_plan_bytes(const wf_round_desc* desc) {
@@ -245,75 +318,16 @@ extern "C" wf_status wf_plan_round(const wf_round_desc* desc, void* host_plan, s
       if (a.pair != b.pair) return a.pair < b.pair;
       return a.part < b.part;
     });
-    // Greedy start: each unit, longest first, to the least-loaded bin
-    // (lowest index on ties).
-    using Bin = std::pair<int64_t, int32_t>;  // (load, index): min-heap pops lowest load, then index
-    std::priority_queue<Bin, std::vector<Bin>, std::greater<Bin>> heap;
-    for (int32_t c = 0; c < g.G; ++c) heap.push({0, c});
-    std::vector<std::vector<wf_plan_unit>> bins(g.G);
-    std::vector<int64_t> load(g.G, 0);
-    for (size_t u = 0; u < units.size(); ++u) {
-      Bin b = heap.top();
-      heap.pop();
-      bins[b.second].push_back(units[u]);
-      load[b.second] += units[u].cost;
-      heap.push({load[b.second], b.second});
-    }
-    // Refinement: with ~6 large units per bin the greedy start leaves the
-    // heaviest bin ~10% above the mean.  Repeatedly move one unit out of the
-    // heaviest bin, or swap it for a lighter one, choosing the change that
-    // leaves the two bins' larger load smallest, from the lightest bin that
-    // offers any change lowering the maximum.  Deterministic: ties keep the
-    // first candidate in bin order, item order, move before swap.
-    for (int iter = 0; iter < 5000; ++iter) {
-      int32_t h = 0;
-      for (int32_t c = 1; c < g.G; ++c)
-        if (load[c] > load[h]) h = c;
-      std::vector<int32_t> order(g.G);
-      for (int32_t c = 0; c < g.G; ++c) order[c] = c;
-      std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return load[a] < load[b]; });
-      int64_t best = -1;
-      int32_t best_b = -1, best_x = -1, best_y = -1;
-      for (int32_t b : order) {
-        if (b == h) continue;
-        if (load[b] >= load[h]) break;
-        for (int32_t xi = 0; xi < int32_t(bins[h].size()); ++xi) {
-          const int64_t x = bins[h][xi].cost;
-          const int64_t mv = std::max(load[h] - x, load[b] + x);
-          if (mv < load[h] && (best < 0 || mv < best)) {
-            best = mv; best_b = b; best_x = xi; best_y = -1;
-          }
-          for (int32_t yi = 0; yi < int32_t(bins[b].size()); ++yi) {
-            const int64_t d = x - bins[b][yi].cost;
-            if (d <= 0) continue;
-            const int64_t sw = std::max(load[h] - d, load[b] + d);
-            if (sw < load[h] && (best < 0 || sw < best)) {
-              best = sw; best_b = b; best_x = xi; best_y = yi;
-            }
-          }
-        }
-        if (best >= 0) break;
-      }
-      if (best < 0) break;
-      const wf_plan_unit x = bins[h][best_x];
-      bins[h].erase(bins[h].begin() + best_x);
-      load[h] -= x.cost;
-      if (best_y >= 0) {
-        const wf_plan_unit y = bins[best_b][best_y];
-        bins[best_b].erase(bins[best_b].begin() + best_y);
-        load[best_b] -= y.cost;
-        bins[h].push_back(y);
-        load[h] += y.cost;
-      }
-      bins[best_b].push_back(x);
-      load[best_b] += x.cost;
-    }
+    std::vector<int64_t> cost(units.size());
+    for (size_t u = 0; u < units.size(); ++u) cost[u] = units[u].cost;
+    std::vector<std::vector<int32_t>> bins;
+    balance(cost, g.G, bins);
     int32_t* cta = reinterpret_cast<int32_t*>(base + g.off_cta);
     wf_plan_unit* out = reinterpret_cast<wf_plan_unit*>(base + g.off_units);
     cta[0] = 0;
     for (int32_t c = 0; c < g.G; ++c) {
       cta[c + 1] = cta[c] + int32_t(bins[c].size());
-      for (size_t k = 0; k < bins[c].size(); ++k) out[cta[c] + k] = bins[c][k];
+      for (size_t k = 0; k < bins[c].size(); ++k) out[cta[c] + k] = units[size_t(bins[c][k])];
     }
   }
 
@@ -323,6 +337,23 @@ extern "C" wf_status wf_plan_round(const wf_round_desc* desc, void* host_plan, s
       cudaGetLastError();
       return WF_ERR_CUDA;
     }
+  }
+  return WF_OK;
+}
+
+extern "C" wf_status wf_balance_units(const int64_t* cost, int32_t n, int32_t bins, int32_t* bin_start,
+                                      int32_t* items) {
+  if (n < 0 || bins < 1 || bins > 65536 || n > (int32_t(1) << 26)) return WF_ERR_INVALID_ARG;
+  if (!bin_start || (n > 0 && (!cost || !items))) return WF_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i)
+    if (cost[i] < 0 || cost[i] > (int64_t(1) << 40)) return WF_ERR_INVALID_ARG;
+  std::vector<int64_t> c(cost, cost + n);
+  std::vector<std::vector<int32_t>> out;
+  balance(c, bins, out);
+  bin_start[0] = 0;
+  for (int32_t b = 0; b < bins; ++b) {
+    bin_start[b + 1] = bin_start[b] + int32_t(out[b].size());
+    for (size_t k = 0; k < out[b].size(); ++k) items[bin_start[b] + int32_t(k)] = out[b][k];
   }
   return WF_OK;
 }

@@ -29,7 +29,7 @@ WF_ATTN_STATUS_BYTES = 256
 WF_FP8_Q, WF_FP8_K = 0, 1
 
 # exported symbols, in the order include/wf.h and include/wf_synth.h declare them
-EXPORTS = ("wf_plan_bytes", "wf_plan_round", "wf_rope3d_append", "wf_attn_workspace_bytes",
+EXPORTS = ("wf_plan_bytes", "wf_plan_round", "wf_balance_units", "wf_rope3d_append", "wf_attn_workspace_bytes",
            "wf_attn_workspace_init", "wf_attn_workspace_status", "wf_chunk_causal_attn",
            "wf_chunk_causal_attn_noalloc", "wf_quantize_fp8", "wf_chunk_causal_attn_fp8", "wf_status_string",
            "wf_version", "wf_synth_fill")
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         dp = ctypes.POINTER(RoundDesc)
         L.wf_plan_bytes.argtypes, L.wf_plan_bytes.restype = [dp], sz
         L.wf_plan_round.argtypes, L.wf_plan_round.restype = [dp, vp, sz, vp, sz, vp], i32
+        L.wf_balance_units.argtypes, L.wf_balance_units.restype = [vp, i32, i32, vp, vp], i32
         L.wf_rope3d_append.argtypes, L.wf_rope3d_append.restype = [vp] * 8 + [vp], i32
         L.wf_attn_workspace_bytes.argtypes, L.wf_attn_workspace_bytes.restype = [vp], sz
         L.wf_attn_workspace_init.argtypes, L.wf_attn_workspace_init.restype = [vp, sz, vp], i32
@@ -144,6 +145,16 @@ def wf_plan_round(desc: RoundDesc, host_plan, dev_plan=None, stream=None, host_b
     db = dev_bytes if dev_bytes is not None else (_nbytes(dev_plan) if dev_plan is not None else 0)
     _check(lib().wf_plan_round(ctypes.byref(desc), _ptr(host_plan), hb, _ptr(dev_plan), db, _stream(stream)),
            "wf_plan_round")
+
+
+def wf_balance_units(costs: Sequence[int], bins: int):
+    """Per bin, the item indices the library's work balancer assigns to it, in list order."""
+    cost = np.ascontiguousarray(np.asarray(costs, dtype=np.int64).reshape(-1))
+    start = np.zeros(bins + 1, dtype=np.int32)
+    items = np.zeros(max(len(cost), 1), dtype=np.int32)
+    _check(lib().wf_balance_units(cost.ctypes.data, len(cost), bins, start.ctypes.data, items.ctypes.data),
+           "wf_balance_units")
+    return [items[start[b]:start[b + 1]].tolist() for b in range(bins)]
 
 
 def wf_rope3d_append(host_plan, dev_plan, q, k, v, q_rot, k_pool, v_pool, stream=None):

@@ -127,6 +127,37 @@ wf_status wf_plan_round(const wf_round_desc* desc, void* host_plan, size_t host_
                         void* dev_plan, size_t dev_bytes, wf_stream_t stream);
 
 /*
+ * wf_balance_units -- the work balancer wf_plan_round applies to the
+ * attention units (its work list is part of the plan), on a given list of
+ * item costs.  The pages describe no scheduler: this is the library's own
+ * rule, exported so that callers (and tests) can check the assignment.
+ *
+ * 1. Longest first: items ordered by cost, largest first (equal costs keep
+ *    their given order), each go to the bin with the smallest load (lowest
+ *    bin index on equal loads).
+ * 2. Refinement, at most 5000 times: h = the heaviest bin (lowest index on
+ *    equal loads).  Scan the other bins from the lightest (lowest index on
+ *    equal loads), stopping at the first that is not lighter than h.  In bin
+ *    b, for each item x of h in list order: moving x gives the larger load
+ *    max(L_h - c_x, L_b + c_x); then for each item y of b in list order with
+ *    c_y < c_x, swapping gives max(L_h - d, L_b + d), d = c_x - c_y.  A change
+ *    counts if that value is below L_h; the best is the smallest value, ties
+ *    to the first found.  The first bin b that offers any change is taken:
+ *    x moves to the end of b's list (and y, for a swap, to the end of h's).
+ *    Stop when no bin offers a change.
+ *
+ * cost:      n item costs, each in [0, 2^40] (host memory).
+ * n:         item count in [0, 2^26].
+ * bins:      bin count in [1, 65536].
+ * bin_start: host int32 [bins + 1] (written): bin b holds items
+ *            items[bin_start[b] .. bin_start[b+1]).
+ * items:     host int32 [n] (written): item indices (into cost), per bin in
+ *            list order.
+ * Errors: WF_ERR_INVALID_ARG (counts, a negative cost, NULL).  Host only.
+ */
+wf_status wf_balance_units(const int64_t* cost, int32_t n, int32_t bins, int32_t* bin_start, int32_t* items);
+
+/*
  * wf_rope3d_append -- 3D rotary embedding of the new Q and K and append of
  * K'/V into the ring pool (the cache write of "scope-causal-forcing", "How It
  * Works", step 2, done for every in-round chunk of the round).

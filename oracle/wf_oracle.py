@@ -177,6 +177,68 @@ def key_parts(units_unsplit: int, num_ctas: int, tiles_min: int, split: bool) ->
     return best_p
 
 
+def balance(costs, num_bins: int):
+    """Share items with the given costs out over num_bins bins.
+
+    Longest first: the items, ordered by cost (largest first; equal costs keep
+    their given order), each go to the bin with the smallest load (the lowest
+    bin index on equal loads).  Then, up to 5000 times: take the heaviest bin h
+    (lowest index on equal loads) and look at the other bins from the lightest
+    (lowest index on equal loads), stopping at the first bin that is not
+    lighter than h.  In a bin b, for each item x of h in its order: moving x
+    to b gives the larger load max(L_h - c_x, L_b + c_x); for each item y of b
+    in its order with c_y < c_x, swapping them gives max(L_h - d, L_b + d),
+    d = c_x - c_y.  A change counts if that value is below L_h; the best one
+    is the smallest value, ties going to the first found (move of x before
+    the swaps of x).  The first bin b offering any change is used: x leaves h
+    (and y, for a swap, leaves b); the arriving items are appended to the end
+    of their new bin's list.  Stop when no bin offers a change.
+
+    Returns (bins, loads): per bin the list of item indices in order, and
+    the bins' total costs."""
+    order = sorted(range(len(costs)), key=lambda i: (-costs[i], i))
+    loads = [0] * num_bins
+    bins = [[] for _ in range(num_bins)]
+    for i in order:
+        c = min(range(num_bins), key=lambda k: (loads[k], k))
+        bins[c].append(i)
+        loads[c] += costs[i]
+    for _ in range(5000):
+        h = max(range(num_bins), key=lambda k: (loads[k], -k))
+        best = None
+        for b in sorted(range(num_bins), key=lambda k: (loads[k], k)):
+            if b == h:
+                continue
+            if loads[b] >= loads[h]:
+                break
+            for xi, x in enumerate(bins[h]):
+                mv = max(loads[h] - costs[x], loads[b] + costs[x])
+                if mv < loads[h] and (best is None or mv < best[0]):
+                    best = (mv, b, xi, None)
+                for yi, y in enumerate(bins[b]):
+                    d = costs[x] - costs[y]
+                    if d <= 0:
+                        continue
+                    sw = max(loads[h] - d, loads[b] + d)
+                    if sw < loads[h] and (best is None or sw < best[0]):
+                        best = (sw, b, xi, yi)
+            if best is not None:
+                break
+        if best is None:
+            break
+        _, b, xi, yi = best
+        x = bins[h].pop(xi)
+        loads[h] -= costs[x]
+        if yi is not None:
+            y = bins[b].pop(yi)
+            loads[b] -= costs[y]
+            bins[h].append(y)
+            loads[h] += costs[y]
+        bins[b].append(x)
+        loads[b] += costs[x]
+    return bins, loads
+
+
 def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas, split=None):
     """Re-derive the round plan: per-chunk visibility/slots and the LPT work list.
     split: share units' keys over several parts when units are few (default:
@@ -211,48 +273,8 @@ def plan_round(H, D, fh, fw, F, Wc, R, S, n0, noise_t, num_ctas, split=None):
                     slot = ((i * H + h) * pairs + p) * P + k if P > 1 else -1
                     units.append((i, h, p, tiles * (9 + live), k, P, slot))
     units.sort(key=lambda u: (-u[3], -u[0], u[1], u[2], u[4]))
-    loads = [0] * num_ctas
-    per_cta = [[] for _ in range(num_ctas)]
-    for u in units:
-        c = min(range(num_ctas), key=lambda k: (loads[k], k))
-        per_cta[c].append(u)
-        loads[c] += u[3]
-    # refinement: move one unit out of the heaviest bin, or swap it for a
-    # lighter one, while that lowers the maximum; best change from the lightest
-    # bin offering any, ties to the first candidate (bin, item, move, swap)
-    for _ in range(5000):
-        h = max(range(num_ctas), key=lambda k: (loads[k], -k))
-        best = None
-        for b in sorted(range(num_ctas), key=lambda k: (loads[k], k)):
-            if b == h:
-                continue
-            if loads[b] >= loads[h]:
-                break
-            for xi, x in enumerate(per_cta[h]):
-                mv = max(loads[h] - x[3], loads[b] + x[3])
-                if mv < loads[h] and (best is None or mv < best[0]):
-                    best = (mv, b, xi, None)
-                for yi, y in enumerate(per_cta[b]):
-                    d = x[3] - y[3]
-                    if d <= 0:
-                        continue
-                    sw = max(loads[h] - d, loads[b] + d)
-                    if sw < loads[h] and (best is None or sw < best[0]):
-                        best = (sw, b, xi, yi)
-            if best is not None:
-                break
-        if best is None:
-            break
-        _, b, xi, yi = best
-        x = per_cta[h].pop(xi)
-        loads[h] -= x[3]
-        if yi is not None:
-            y = per_cta[b].pop(yi)
-            loads[b] -= y[3]
-            per_cta[h].append(y)
-            loads[h] += y[3]
-        per_cta[b].append(x)
-        loads[b] += x[3]
+    bins, loads = balance([u[3] for u in units], num_ctas)
+    per_cta = [[units[k] for k in b] for b in bins]
     return dict(C=C, wc_eff=wc_eff, first=first, chunks=chunks, units=units,
                 per_cta=per_cta, loads=loads, q_pairs=pairs, key_parts=P)
 

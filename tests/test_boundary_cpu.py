@@ -218,6 +218,27 @@ def test_plan_golden_cases_through_the_library():
             assert [[list(u[:3]) for u in lst] for lst in p["per_cta"]] == c["per_cta"]
 
 
+def test_balance_golden_cases_through_the_library():
+    for c in json.load(open(os.path.join(GOLDEN, "balance_cases.json")))["cases"]:
+        assert wf.wf_balance_units(c["costs"], c["num_bins"]) == c["bins"], c["name"]
+
+
+def test_balance_library_matches_oracle_on_random_lists():
+    rng = np.random.default_rng(11)
+    for _ in range(400):
+        n = int(rng.integers(0, 40))
+        G = int(rng.integers(1, 9))
+        costs = [int(x) for x in rng.integers(0, int(rng.choice([3, 20, 1000])), n)]
+        assert wf.wf_balance_units(costs, G) == orc.balance(costs, G)[0], (costs, G)
+
+
+@pytest.mark.parametrize("costs,bins", [([1, -1], 2), ([1, 2], 0), ([1], 65537), ([1 << 41], 2)])
+def test_balance_rejects_bad_arguments(costs, bins):
+    with pytest.raises(wf.WfError) as e:
+        wf.wf_balance_units(costs, bins)
+    assert e.value.code == wf.WF_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("D,pairs", [(64, (0, 0, 0)), (128, (0, 0, 0)), (64, (11, 11, 10)), (128, (64, 0, 0))])
 def test_plan_rope_tables_match_oracle_angles(D, pairs):
     dtype = wf.WF_BF16 if D == 128 else wf.WF_F32

@@ -192,6 +192,41 @@ def test_plan_golden_cases():
             assert p["loads"] == c["loads"]
 
 
+def test_balance_golden_cases():
+    """Hand-derived assignments of the work balancer, one per tie-break and branch."""
+    for c in load("balance_cases.json")["cases"]:
+        bins, loads = orc.balance(c["costs"], c["num_bins"])
+        assert bins == c["bins"], c["name"]
+        assert loads == c["loads"], c["name"]
+
+
+def test_balance_leaves_no_improving_move_or_swap():
+    """On random cost lists: the result is a partition of the items, and no move or
+    swap between the heaviest bin and a lighter one lowers the heaviest load (the
+    refinement's stopping condition, checked by brute force)."""
+    rng = np.random.default_rng(7)
+    for _ in range(300):
+        n = int(rng.integers(0, 14))
+        G = int(rng.integers(1, 6))
+        costs = [int(x) for x in rng.integers(0, 40, n)]
+        bins, loads = orc.balance(costs, G)
+        assert sorted(i for b in bins for i in b) == list(range(n))
+        assert loads == [sum(costs[i] for i in b) for b in bins]
+        top = max(loads)
+        for h in range(G):
+            if loads[h] != top:
+                continue
+            for b in range(G):
+                if loads[b] >= top:
+                    continue
+                for x in bins[h]:
+                    assert max(top - costs[x], loads[b] + costs[x]) >= top
+                    for y in bins[b]:
+                        d = costs[x] - costs[y]
+                        assert d <= 0 or max(top - d, loads[b] + d) >= top
+            break
+
+
 def test_plan_tile_pairs_match_brute_mask():
     """Key tiles the plan visits per query chunk cover exactly the visible keys."""
     for (C, Wc, R, S, n0) in [(48, 3, 3, 6, 3), (48, 3, 3, 6, 5), (200, 2, 4, 6, 9), (130, 0, 2, 2, 4)]:
