@@ -366,9 +366,12 @@ def fp8_block_quantize(x, C: int):
     """x: [n*C, H, D] values (exact in fp32), n whole chunks of C tokens.
 
     Per chunk, block b of tokens [b*FP8_BLOCK, min(C, (b+1)*FP8_BLOCK)) and
-    head: scale = fp32(amax / 448), inv = fp32(448 / amax) (both 1 for an
-    all-zero block), codes = round_e4m3(fp32(x * inv)).  Every fp32
-    operation is a single operation rounded to nearest.  Returns (codes
+    head: scale = fp32(amax / 448), inv = fp32(448 / amax), codes =
+    round_e4m3(fp32(x * inv)).  Every fp32 operation is a single operation
+    rounded to nearest.  A block whose fp32 448 / amax is not finite (amax =
+    0, or amax below 448 / FLT_MAX ~ 1.3e-36) is treated as all-zero: scale
+    and inv are 1, so its elements round to zero codes (an infinite inv would
+    turn every zero into 0 * inf = NaN).  Returns (codes
     [n*C, H, D] as values, scales [n, nblk, H] float64 holding fp32 values).
     """
     x = np.asarray(x, dtype=np.float64)
@@ -382,10 +385,12 @@ def fp8_block_quantize(x, C: int):
             lo, hi = c * C + b * FP8_BLOCK, c * C + min(C, (b + 1) * FP8_BLOCK)
             blk = x[lo:hi].astype(np.float32)                       # [tokens, H, D], exact
             amax = np.abs(blk).max(axis=(0, 2))                      # [H]
-            nz = amax > 0
-            safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
-            sc = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-            inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
+            safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+            with np.errstate(over="ignore"):
+                inv_raw = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+            ok = (amax > 0) & np.isfinite(inv_raw)
+            sc = np.where(ok, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+            inv = np.where(ok, inv_raw, np.float32(1.0)).astype(np.float32)
             scales[c, b] = sc
             codes[lo:hi] = round_e4m3((blk * inv[None, :, None]).astype(np.float32))
     return codes, scales

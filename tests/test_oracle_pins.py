@@ -495,6 +495,22 @@ def test_fp8_block_quantize_hand_case():
     assert np.array_equal(deq[5, 0], x[5, 0]) and np.array_equal(deq[70, 0], x[70, 0])
 
 
+def test_fp8_block_quantize_tiny_block_is_a_zero_block():
+    # a block of zeros plus one bf16 subnormal (2^-133): 448 / 2^-133 overflows fp32, so the
+    # block takes scale 1 and inv 1 like an all-zero block, and every code is zero -- no NaN
+    # from 0 * inf.  A block whose amax (2^-100) keeps 448 / amax finite is quantized as usual.
+    C, H, D = 128, 2, 4
+    x = np.zeros((C, H, D))
+    x[7, 0, 2] = 2.0 ** -133
+    x[9, 0, 1] = -2.0 ** -133
+    x[3, 1, 0] = 2.0 ** -100
+    codes, scales = orc.fp8_block_quantize(x, C)
+    assert scales[0, 0, 0] == 1.0 and not np.isnan(codes).any()
+    assert np.array_equal(codes[:, 0], np.zeros((C, D)))
+    assert scales[0, 0, 1] == float(np.float32(2.0 ** -100) / np.float32(448.0))
+    assert codes[3, 1, 0] == 448.0
+
+
 def test_fp8_dequantized_error_within_half_an_e4m3_step():
     rng = np.random.default_rng(3)
     C = 300
