@@ -85,8 +85,12 @@ __global__ void __launch_bounds__(256, 4) fp8_quant_kernel(const QuantParams p) 
   amax = warp_max[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
-  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  // a block whose 448 / amax is not finite (amax 0 or below 448 / FLT_MAX) is
+  // an all-zero block: scale 1, inv 1 (an infinite inv would give 0 * inf = NaN)
+  const float inv_raw = __fdiv_rn(448.0f, amax);
+  const bool regular = amax > 0.f && isfinite(inv_raw);
+  const float scale = regular ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const float inv = regular ? inv_raw : 1.0f;
 #pragma unroll
   for (int s = 0; s < kPasses; ++s) {
     const int r = s * kRowsPerPass + r0;

@@ -16,6 +16,7 @@ import torch
 
 from chunk_causal_attention_block_b200 import wf
 from chunk_causal_attention_block_b200.rollout import CONFIGS, RoundConfig
+from oracle import wf_oracle as orc
 from tests import gpu_common as gc
 
 pytestmark = pytest.mark.gpu
@@ -177,3 +178,30 @@ def test_negative_controls_fail_the_gates():
     keep[: 3 * n_keys // 4] = True
     with pytest.raises(AssertionError):
         gc.assert_bf16_close(got, attend(k, v, mask & keep[None, :]), "a key part dropped")
+
+
+def test_fp8_quantize_tiny_and_zero_blocks_bit_exact():
+    """Blocks whose 448 / amax overflows fp32 (zeros plus bf16 subnormals) quantize like all-zero
+    blocks (scale 1, zero codes, no NaN), next to a normal block and an all-zero one; codes and
+    scales bit-exact against the oracle."""
+    C, H, D, R = 256, 4, 128, 1
+    desc = wf.make_desc(H, D, 1, C, 1, 0, R, 0, [1000], dtype=wf.WF_BF16, num_ctas=2)
+    host = wf.host_plan_buffer(desc)
+    dev = torch.empty(host.numel(), dtype=torch.uint8, device="cuda")
+    wf.wf_plan_round(desc, host, dev)
+    x = torch.zeros(R * C, H, D, dtype=torch.float64)
+    x[5, 0, 7] = 2.0 ** -133                   # head 0, block 0: one subnormal
+    x[200, 0, 3] = -(2.0 ** -126)              # head 0, block 1: amax 2^-126, still overflows
+    x[17, 1, 9] = 2.0 ** -100                  # head 1, block 0: tiny but regular
+    x[:, 2] = torch.linspace(-3, 3, R * C * D, dtype=torch.float64).reshape(R * C, D)  # head 2: normal
+    src = x.to(torch.bfloat16).cuda()          # head 3 stays all-zero
+    dst = torch.full((R * C, H, D), 0x7F, dtype=torch.uint8, device="cuda")
+    scales = torch.full((R, 2, H), float("nan"), dtype=torch.float32, device="cuda")
+    wf.wf_quantize_fp8(host, src, dst, scales, wf.WF_FP8_Q)
+    torch.cuda.synchronize()
+    codes, ref_scales = orc.fp8_block_quantize(src.float().cpu().numpy().astype(np.float64), C)
+    got = _e4m3_values(dst)
+    assert not np.isnan(got).any()
+    assert np.array_equal(got, codes)
+    assert np.array_equal(scales.cpu().numpy().astype(np.float64), ref_scales)
+    assert (ref_scales[0, :, 0] == 1.0).all() and not codes[:, 0].any()
