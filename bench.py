@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--config", default="wan13b_round")
     ap.add_argument("--scores", choices=("bf16", "fp8"), default="bf16",
                     help="fp8: e4m3 Q/K codes with block scales (quantization timed with RoPE/append)")
+    ap.add_argument("--fused-q-rope", action="store_true",
+                    help="the attention rotates the raw Q itself; the append pass writes only K'/V")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -64,7 +66,7 @@ def kernel_source_sha(read=None):
     """Hash of the attention kernel's code (line comments and blank lines
     dropped, so that editing a comment does not orphan a capture)."""
     h = hashlib.sha256()
-    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "wf_plan.h", "wf_plan.cpp"):
+    for name in ("attn_sm100.cu", "sm100_ptx.cuh", "rope_math.cuh", "wf_plan.h", "wf_plan.cpp"):
         if read is None:
             with open(os.path.join(ROOT, "chunk_causal_attention_block_b200", "csrc", name)) as f:
                 text = f.read()
@@ -239,7 +241,8 @@ def run_wf(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     W, K = args.warmup, args.steps
-    ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank), fp8=args.scores == "fp8")
+    ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank), fp8=args.scores == "fp8",
+                 fused_q_rope=args.fused_q_rope)
     ro.prefill()
 
     # every step's inputs resident in HBM before timing (round r draws tag r)
@@ -396,6 +399,8 @@ def run_wf(args, rank, world, local_rank):
     flops = cfg.attn_flops()
     attn_avg = statistics.mean(attn_ms)
     rope_avg = statistics.mean(rope_ms)
+    # the append pass moves Q, K, V in and Q', K', V out; K and V only when Q's RoPE is fused
+    rope_bytes = cfg.rope_bytes() * (4 if args.fused_q_rope else 6) // 6
     achieved = flops / (attn_avg / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic = dram_traffic(args.config)
@@ -427,9 +432,9 @@ def run_wf(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "attn_fwd_sm100", "peak_kind": f"{peak_kind} bf16 burst"},
-        "rope_append": {"ms": rope_avg, "gb_s": cfg.rope_bytes() / (rope_avg / 1e3) / 1e9,
-                        "frac_of_hbm": cfg.rope_bytes() / (rope_avg / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
-                        "bytes": cfg.rope_bytes()},
+        "rope_append": {"ms": rope_avg, "gb_s": rope_bytes / (rope_avg / 1e3) / 1e9,
+                        "frac_of_hbm": rope_bytes / (rope_avg / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+                        "bytes": rope_bytes, "fused_q_rope": args.fused_q_rope},
         "attn_ms": attn_avg,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,

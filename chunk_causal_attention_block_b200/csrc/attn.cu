@@ -23,6 +23,9 @@ namespace wf {
 wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_rot, const void* k_pool,
                             const void* v_pool, void* out, float* lse, float scale, void* workspace,
                             uint64_t timeout_ns, cudaStream_t stream);
+wf_status launch_attn_sm100_rope_q(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_raw,
+                                   const void* k_pool, const void* v_pool, void* out, float* lse, float scale,
+                                   void* workspace, uint64_t timeout_ns, cudaStream_t stream);
 wf_status launch_attn_sm100_fp8(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q8, const float* q_scales,
                                 const void* k8_pool, const float* k_scales, const void* v_pool, void* out, float* lse,
                                 float scale, void* workspace, uint64_t timeout_ns, cudaStream_t stream);
@@ -279,6 +282,26 @@ extern "C" wf_status wf_chunk_causal_attn(const void* host_plan, const void* dev
   else
     attn_f32_kernel<128><<<grid, 128, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? WF_OK : WF_ERR_CUDA;
+}
+
+extern "C" wf_status wf_chunk_causal_attn_rope(const void* host_plan, const void* dev_plan, const void* q,
+                                               const void* k_pool, const void* v_pool, void* out, float* lse,
+                                               float softmax_scale, void* workspace, size_t workspace_bytes,
+                                               wf_stream_t stream) {
+  if (!host_plan || !dev_plan || !q || !k_pool || !v_pool || !out || !workspace) return WF_ERR_INVALID_ARG;
+  const wf_plan_hdr* h = static_cast<const wf_plan_hdr*>(host_plan);
+  if (h->magic != WF_PLAN_MAGIC || h->version != WF_PLAN_VERSION) return WF_ERR_PLAN;
+  if (misaligned(dev_plan) || misaligned(q) || misaligned(k_pool) || misaligned(v_pool) || misaligned(out) ||
+      misaligned(workspace) || (reinterpret_cast<uintptr_t>(lse) % 4))
+    return WF_ERR_ALIGNMENT;
+  if (workspace_bytes < wf_attn_workspace_bytes(host_plan)) return WF_ERR_WORKSPACE;
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return WF_ERR_INVALID_ARG;
+  if (h->dtype != WF_BF16 || h->D != 128) return WF_ERR_UNSUPPORTED;
+  const float scale = softmax_scale == 0.f ? float(1.0 / std::sqrt(double(h->D))) : softmax_scale;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const wf_status st = wf::launch_attn_sm100_rope_q(h, static_cast<const uint8_t*>(dev_plan), q, k_pool, v_pool, out,
+                                                    lse, scale, workspace, wait_timeout_ns(), s);
+  return st == WF_OK ? launch_combine(h, host_plan, workspace, out, lse, s) : st;
 }
 
 extern "C" wf_status wf_chunk_causal_attn_fp8(const void* host_plan, const void* dev_plan, const void* q8,

@@ -47,10 +47,12 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
 
+#include "rope_math.cuh"
 #include "sm100_ptx.cuh"
 #include "wf.h"
 #include "wf_plan.h"
@@ -58,14 +60,12 @@
 namespace wf {
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kThreads = 384;
 constexpr uint32_t kSoftmaxRegs = 224;
 constexpr uint32_t kControlRegs = 56;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * 168, "register split must match launch");
 constexpr int kTileBytes = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr int kHalfBytes = kTileBytes / 2; // one 64-column (128-byte) half
-constexpr int kSmemBytes = 1024 + 2 * kTileBytes + kStages * kTileBytes + 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -94,39 +94,72 @@ struct Params {
   // split units: normalised partial O [slot][256][128] and LSE [slot][256]
   float* part_o;
   float* part_lse;
+  // Q's RoPE in the kernel: the device plan (token grid, fp64 (cos, sin) tables).
+  // Read from the plan rather than passed here: a larger parameter block made
+  // ptxas spill in the softmax.
+  const wf_plan_hdr* plan;
 };
 
-// Barrier indices in the barrier block.
-enum : int {
-  kBarQFull = 0,
-  kBarQEmpty = 1,
-  kBarSFull = 2,     // +t
-  kBarPFull = 4,     // +t
-  kBarOFull = 6,     // +t
-  kBarMmaDone = 8,
-  kBarKVFull = 9,    // +stage
-  kBarKVEmpty = 9 + kStages,
-  kNumBars = 9 + 2 * kStages
+// Token grid and table offsets for the in-kernel Q rotation, copied from the
+// plan into shared memory (re-read there each row: held in registers across
+// the loop they pushed the 56-register control warps into spills).
+struct RopeConsts {
+  uint32_t fw, fhw, F;
+  int32_t Pt, Ph, Pw;
+  uint32_t off_t, off_h, off_w;
+};
+
+// Shared-memory and barrier layout.  The kRopeQ instantiation (Q's RoPE done
+// in the kernel) double-buffers Q so that the next unit's tile can be rotated
+// while the current unit runs, and keeps three K/V stages to stay within
+// 227 KB; the others hold one Q buffer and four K/V stages.
+template <bool kRopeQ>
+struct Layout {
+  static constexpr int kQBufs = kRopeQ ? 2 : 1;
+  static constexpr int kStages = kRopeQ ? 3 : 4;
+  static constexpr int kQFull = 0;                             // + buffer: Q ready for the MMAs
+  static constexpr int kQEmpty = kQFull + kQBufs;              // + buffer: last S MMA of its unit done
+  static constexpr int kQRaw = kQEmpty + kQBufs;               // + buffer: raw Q landed (kRopeQ)
+  static constexpr int kSFull = kQRaw + (kRopeQ ? kQBufs : 0);  // + t
+  static constexpr int kPFull = kSFull + 2;                    // + t
+  static constexpr int kOFull = kPFull + 2;                    // + t
+  static constexpr int kMmaDone = kOFull + 2;
+  static constexpr int kKVFull = kMmaDone + 1;                 // + stage
+  static constexpr int kKVEmpty = kKVFull + kStages;           // + stage
+  static constexpr int kNumBars = kKVEmpty + kStages;
+  static constexpr int kTiles = 2 * kQBufs + kStages;          // 32 KB tiles: Q buffers, then K/V stages
+  static constexpr int kSmemBytes = 1024 + kTiles * kTileBytes + 256;
+  static_assert(8 * kNumBars + 8 + sizeof(RopeConsts) <= 256, "barrier block");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
 struct Shared {
-  uint8_t* base;  // Q_0 | Q_1 | K/V stages, each kTileBytes, 1024-aligned
+  uint8_t* base;  // Q buffers (two tiles each), then the K/V stages; 1024-aligned
   uint64_t* bars;
   uint32_t* tmem_slot;
   int32_t* abort_flag;
+  RopeConsts* rope;
 };
 
-__device__ __forceinline__ uint8_t* q_tile(const Shared& s, int t) { return s.base + t * kTileBytes; }
-__device__ __forceinline__ uint8_t* kv_tile(const Shared& s, int st) { return s.base + (2 + st) * kTileBytes; }
+template <bool kRopeQ>
+__device__ __forceinline__ uint8_t* q_tile(const Shared& s, int buf, int t) {
+  return s.base + (2 * buf + t) * kTileBytes;
+}
+template <bool kRopeQ>
+__device__ __forceinline__ uint8_t* kv_tile(const Shared& s, int st) {
+  return s.base + (2 * Layout<kRopeQ>::kQBufs + st) * kTileBytes;
+}
 
+template <bool kRopeQ>
 __device__ __forceinline__ Shared carve_smem(uint8_t* raw) {
   Shared s;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.base = base;
-  uint8_t* tail = base + (2 + kStages) * kTileBytes;
+  uint8_t* tail = base + Layout<kRopeQ>::kTiles * kTileBytes;
   s.bars = reinterpret_cast<uint64_t*>(tail);
-  s.tmem_slot = reinterpret_cast<uint32_t*>(tail + 8 * kNumBars);
-  s.abort_flag = reinterpret_cast<int32_t*>(tail + 8 * kNumBars + 4);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(tail + 8 * Layout<kRopeQ>::kNumBars);
+  s.abort_flag = reinterpret_cast<int32_t*>(tail + 8 * Layout<kRopeQ>::kNumBars + 4);
+  s.rope = reinterpret_cast<RopeConsts*>(tail + 8 * Layout<kRopeQ>::kNumBars + 8);
   return s;
 }
 
@@ -213,37 +246,62 @@ __device__ __forceinline__ wf_plan_chunk load_chunk(const wf_plan_chunk* p) {
 
 // ---------------------------------------------------------------- roles
 
-template <bool kFp8>
-__device__ __forceinline__ void producer(const Shared& sh, const Params& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                         const CUtensorMap* tm_v, int u0, int u1) {
+// TMA loads of one unit's query tiles into Q buffer `buf`, completing on `bar`
+// (the raw tiles when the kernel rotates Q itself).
+template <bool kFp8, bool kRopeQ>
+__device__ __forceinline__ void load_q(const Shared& sh, const CUtensorMap* tm_q, const wf_plan_unit& unit, int C,
+                                       int buf, uint32_t bar) {
+  const int32_t row0 = unit.chunk * C + unit.pair * 256;
+  const bool live1 = C - unit.pair * 256 > 128;
+  uint8_t* q0 = q_tile<kRopeQ>(sh, buf, 0);
+  uint8_t* q1 = q_tile<kRopeQ>(sh, buf, 1);
+  if constexpr (kFp8) {
+    mbar_arrive_expect_tx(bar, live1 ? 2 * kTile8Bytes : kTile8Bytes);
+    tma_load_3d(smem_u32(q0), tm_q, bar, 0, unit.head, row0);
+    if (live1) tma_load_3d(smem_u32(q1), tm_q, bar, 0, unit.head, row0 + 128);
+  } else {
+    mbar_arrive_expect_tx(bar, live1 ? 2 * kTileBytes : kTileBytes);
+    tma_load_3d(smem_u32(q0), tm_q, bar, 0, unit.head, row0);
+    tma_load_3d(smem_u32(q0 + kHalfBytes), tm_q, bar, 64, unit.head, row0);
+    if (live1) {
+      tma_load_3d(smem_u32(q1), tm_q, bar, 0, unit.head, row0 + 128);
+      tma_load_3d(smem_u32(q1 + kHalfBytes), tm_q, bar, 64, unit.head, row0 + 128);
+    }
+  }
+}
+
+template <bool kFp8, bool kRopeQ>
+__device__ __forceinline__ void producer(const Shared& sh, const Params& p, const CUtensorMap* tm_q,
+                                         const CUtensorMap* tm_k, const CUtensorMap* tm_v, int u0, int u1) {
+  using L = Layout<kRopeQ>;
+  constexpr int kQB = L::kQBufs;
   int kv_it = 0;
-  int q_it = 0;
+  int q_it = 0;  // Q loads issued
   bool ok = true;
+  // Q load of unit u into buffer q_it % kQB, once the unit that last used
+  // that buffer has issued its final score MMA.
+  auto issue_q = [&](int u) -> bool {
+    const int buf = q_it % kQB;
+    if (q_it >= kQB && !wait_bar(sh, p, L::kQEmpty + buf, ((q_it / kQB) - 1) & 1, 1)) return false;
+    const uint32_t bar = smem_u32(sh.bars + (kRopeQ ? L::kQRaw : L::kQFull) + buf);
+    load_q<kFp8, kRopeQ>(sh, tm_q, p.units[u], p.C, buf, bar);
+    ++q_it;
+    return true;
+  };
+  if (kRopeQ && u0 < u1 && !issue_q(u0)) ok = false;
   for (int u = u0; u < u1 && ok; ++u) {
     const wf_plan_unit unit = p.units[u];
     const wf_plan_chunk c = load_chunk(p.chunks + unit.chunk);
-    const int32_t row0 = unit.chunk * p.C + unit.pair * 256;
-    const bool live1 = p.C - unit.pair * 256 > 128;
-    if (q_it > 0 && !wait_bar(sh, p, kBarQEmpty, (q_it - 1) & 1, 1)) { ok = false; break; }
-    const uint32_t qbar = smem_u32(sh.bars + kBarQFull);
-    if constexpr (kFp8) {
-      mbar_arrive_expect_tx(qbar, live1 ? 2 * kTile8Bytes : kTile8Bytes);
-      tma_load_3d(smem_u32(q_tile(sh, 0)), tm_q, qbar, 0, unit.head, row0);
-      if (live1) tma_load_3d(smem_u32(q_tile(sh, 1)), tm_q, qbar, 0, unit.head, row0 + 128);
-    } else {
-      mbar_arrive_expect_tx(qbar, live1 ? 2 * kTileBytes : kTileBytes);
-      tma_load_3d(smem_u32(q_tile(sh, 0)), tm_q, qbar, 0, unit.head, row0);
-      tma_load_3d(smem_u32(q_tile(sh, 0) + kHalfBytes), tm_q, qbar, 64, unit.head, row0);
-      if (live1) {
-        tma_load_3d(smem_u32(q_tile(sh, 1)), tm_q, qbar, 0, unit.head, row0 + 128);
-        tma_load_3d(smem_u32(q_tile(sh, 1) + kHalfBytes), tm_q, qbar, 64, unit.head, row0 + 128);
-      }
-    }
-    ++q_it;
+    if (!kRopeQ && !issue_q(u)) { ok = false; break; }
     const int first_slot = kFp8 ? first_visible_slot(p, p.chunks + unit.chunk) : 0;
     int t0, t1;
     unit_tile_range(unit, unit_key_tiles<kFp8>(p, p.chunks + unit.chunk), t0, t1);
+    // with two Q buffers the next unit's tile is loaded once this unit's
+    // first key tiles are in flight (so the buffer it reuses is surely free
+    // soon), leaving the rotation the rest of this unit to finish
+    const int q_next_at = t0 + (t1 - t0 < L::kStages ? t1 - t0 : L::kStages);
     for (int j = t0; j < t1; ++j) {
+      if (kRopeQ && j == q_next_at && u + 1 < u1 && !issue_q(u + 1)) { ok = false; break; }
       int32_t tok, valid;
       if constexpr (kFp8) {
         int32_t slot, blk;
@@ -253,45 +311,117 @@ __device__ __forceinline__ void producer(const Shared& sh, const Params& p, cons
       }
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
-        const int st = kv_it % kStages;
+        const int st = kv_it % L::kStages;
         if (p.stall_first_load && blockIdx.x == 0 && kv_it == 0) {
           // failure-detection test: this fill's barrier is never armed, so
           // the MMA thread's bounded wait on it must expire
           ++kv_it;
           continue;
         }
-        if (!wait_bar(sh, p, kBarKVEmpty + st, ((kv_it / kStages) & 1) ^ 1, 2)) { ok = false; break; }
-        const uint32_t bar = smem_u32(sh.bars + kBarKVFull + st);
+        if (!wait_bar(sh, p, L::kKVEmpty + st, ((kv_it / L::kStages) & 1) ^ 1, 2)) { ok = false; break; }
+        const uint32_t bar = smem_u32(sh.bars + L::kKVFull + st);
         const CUtensorMap* tm = kv == 0 ? tm_k : tm_v;
+        uint8_t* dst = kv_tile<kRopeQ>(sh, st);
         if (kFp8 && kv == 0) {  // e4m3 K: one 128-byte-wide box
           mbar_arrive_expect_tx(bar, kTile8Bytes);
-          tma_load_3d(smem_u32(kv_tile(sh, st)), tm, bar, 0, unit.head, tok);
+          tma_load_3d(smem_u32(dst), tm, bar, 0, unit.head, tok);
         } else {
           mbar_arrive_expect_tx(bar, kTileBytes);
-          tma_load_3d(smem_u32(kv_tile(sh, st)), tm, bar, 0, unit.head, tok);
-          tma_load_3d(smem_u32(kv_tile(sh, st) + kHalfBytes), tm, bar, 64, unit.head, tok);
+          tma_load_3d(smem_u32(dst), tm, bar, 0, unit.head, tok);
+          tma_load_3d(smem_u32(dst + kHalfBytes), tm, bar, 64, unit.head, tok);
         }
         ++kv_it;
       }
       if (!ok) break;
     }
+    if (ok && kRopeQ && q_next_at >= t1 && u + 1 < u1 && !issue_q(u + 1)) ok = false;
   }
   // Drain: the CTA must not exit with bulk copies still landing in its smem.
   if (!ok) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       if (kv_it <= s) continue;
-      const int last_fill = (kv_it - 1 - s) / kStages;  // fill count - 1 of stage s
-      const uint32_t addr = smem_u32(sh.bars + kBarKVFull + s);
+      const int last_fill = (kv_it - 1 - s) / L::kStages;  // fill count - 1 of stage s
+      const uint32_t addr = smem_u32(sh.bars + L::kKVFull + s);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(addr, uint32_t(last_fill) & 1) && global_timer_ns() - t0 < p.timeout_ns) {
       }
     }
-    if (q_it > 0) {
-      const uint32_t addr = smem_u32(sh.bars + kBarQFull);
+    for (int b = 0; b < kQB; ++b) {
+      if (q_it <= b) continue;
+      const int last_fill = (q_it - 1 - b) / kQB;
+      const uint32_t addr = smem_u32(sh.bars + (kRopeQ ? L::kQRaw : L::kQFull) + b);
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(addr, uint32_t(q_it - 1) & 1) && global_timer_ns() - t0 < p.timeout_ns) {
+      while (!mbar_try_wait(addr, uint32_t(last_fill) & 1) && global_timer_ns() - t0 < p.timeout_ns) {
       }
     }
+  }
+}
+
+// kRopeQ: warps 10-11 rotate each unit's raw query tiles in place, in fp64
+// from the plan's tables, rounding once to bf16 exactly as wf_rope3d_append
+// does, then hand the buffer to the MMA thread.  In the 128-byte-swizzled
+// tile, row r's 16-byte chunk c of a 64-column half sits at chunk c ^ (r % 8);
+// an interleaved pair never straddles a chunk.  Rows past the chunk's end are
+// left as loaded (their outputs are never stored).
+__device__ __forceinline__ void rope_q_role(const Shared& sh, const Params& p, int u0, int u1) {
+  using L = Layout<true>;
+  const int th = threadIdx.x - 320;  // 0..63
+  // 64 threads stride over a tile's 128 rows x 16 chunks: each thread keeps
+  // chunk column cc (dims 8cc..8cc+7, pairs 4cc..4cc+3) on every fourth row
+  const int cc = th & 15;
+  const uint32_t q_base = smem_u32(q_tile<true>(sh, 0, 0)) + (cc >> 3) * kHalfBytes;
+  const uint32_t rc_addr = smem_u32(sh.rope);
+  const uint8_t* plan = reinterpret_cast<const uint8_t*>(p.plan);
+  int q_it = 0;
+  for (int u = u0; u < u1; ++u, ++q_it) {
+    const int buf = q_it % L::kQBufs;
+    if (!__all_sync(0xffffffffu, wait_bar(sh, p, L::kQRaw + buf, (q_it / L::kQBufs) & 1, 30))) return;
+    const int32_t chunk = p.units[u].chunk, pair = p.units[u].pair;
+    for (int t = 0; t < 2; ++t) {
+      const int rows_here = p.C - pair * 256 - 128 * t;
+      if (rows_here <= 0) break;
+      const uint32_t tile = q_base + uint32_t(2 * buf + t) * kTileBytes;
+#pragma unroll 1
+      for (int row = th >> 4; row < 128 && row < rows_here; row += 4) {
+        const uint32_t addr = tile + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
+        const uint32_t fw = ld_shared_u32(rc_addr + offsetof(RopeConsts, fw));
+        const uint32_t fhw = ld_shared_u32(rc_addr + offsetof(RopeConsts, fhw));
+        const uint32_t q = uint32_t(pair * 256 + 128 * t + row);  // token inside the chunk
+        const uint32_t f = q / fhw, l = q - f * fhw;
+        const uint32_t hh = l / fw, ww = l - hh * fw;
+        const uint32_t trow = uint32_t(chunk) * ld_shared_u32(rc_addr + offsetof(RopeConsts, F)) + f;
+        uint32_t w[4];
+        ld_shared_v4(addr, w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int32_t m = 4 * cc + k;
+          const int32_t Pt = int32_t(ld_shared_u32(rc_addr + offsetof(RopeConsts, Pt)));
+          const int32_t Ph = int32_t(ld_shared_u32(rc_addr + offsetof(RopeConsts, Ph)));
+          const double2* tab;
+          if (m < Pt) {
+            tab = reinterpret_cast<const double2*>(plan + ld_shared_u32(rc_addr + offsetof(RopeConsts, off_t))) +
+                  int64_t(trow) * Pt + m;
+          } else if (m < Pt + Ph) {
+            tab = reinterpret_cast<const double2*>(plan + ld_shared_u32(rc_addr + offsetof(RopeConsts, off_h))) +
+                  int64_t(hh) * Ph + (m - Pt);
+          } else {
+            const int32_t Pw = int32_t(ld_shared_u32(rc_addr + offsetof(RopeConsts, Pw)));
+            tab = reinterpret_cast<const double2*>(plan + ld_shared_u32(rc_addr + offsetof(RopeConsts, off_w))) +
+                  int64_t(ww) * Pw + (m - Pt - Ph);
+          }
+          w[k] = rope_pair_bf16(w[k], __ldg(tab));
+        }
+        st_shared_v4(addr, w[0], w[1], w[2], w[3]);
+      }
+    }
+    // make the rotated tile visible to the tensor cores (async proxy)
+    fence_proxy_async_smem();
+#if WF_WARP_ARRIVE
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(sh.bars + L::kQFull + buf));
+#else
+    mbar_arrive(smem_u32(sh.bars + L::kQFull + buf));
+#endif
   }
 }
 
@@ -351,84 +481,130 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, const
   issue_pv_slice<0>(o_tmem, p_tmem, mnmajor_desc(v), accumulate ? 1u : 0u);
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kRopeQ>
 __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, uint32_t tmem, int u0, int u1) {
+  using L = Layout<kRopeQ>;
   int kv_it = 0, q_it = 0;
   int p_cnt[2] = {0, 0};
   bool ok = true;
   const uint32_t s_tm[2] = {tmem + 0, tmem + 128};
   const uint32_t o_tm[2] = {tmem + 256, tmem + 384};
-  const uint64_t qd0 = kmajor_desc(q_tile(sh, 0)), qd1 = kmajor_desc(q_tile(sh, 1));
   for (int u = u0; u < u1 && ok; ++u) {
     const wf_plan_unit unit = p.units[u];
     int t0, t1;
     unit_tile_range(unit, unit_key_tiles<kFp8>(p, p.chunks + unit.chunk), t0, t1);
     const int n = t1 - t0;  // key tiles of this unit
     const bool live1 = p.C - unit.pair * 256 > 128;
-    if (!wait_bar(sh, p, kBarQFull, q_it & 1, 10)) { ok = false; break; }
+    const int qbuf = q_it % L::kQBufs;
+    if (!wait_bar(sh, p, L::kQFull + qbuf, (q_it / L::kQBufs) & 1, 10)) { ok = false; break; }
     ++q_it;
+    const uint64_t qd0 = kmajor_desc(q_tile<kRopeQ>(sh, qbuf, 0)), qd1 = kmajor_desc(q_tile<kRopeQ>(sh, qbuf, 1));
     tc_fence_after();
-    int kst = kv_it % kStages;
-    if (!wait_bar(sh, p, kBarKVFull + kst, (kv_it / kStages) & 1, 11)) { ok = false; break; }
+    int kst = kv_it % L::kStages;
+    if (!wait_bar(sh, p, L::kKVFull + kst, (kv_it / L::kStages) & 1, 11)) { ok = false; break; }
     ++kv_it;
     tc_fence_after();
-    issue_s<kFp8>(s_tm[0], qd0, kv_tile(sh, kst));
-    mma_commit(smem_u32(sh.bars + kBarSFull + 0));
+    issue_s<kFp8>(s_tm[0], qd0, kv_tile<kRopeQ>(sh, kst));
+    mma_commit(smem_u32(sh.bars + L::kSFull + 0));
     if (live1) {
-      issue_s<kFp8>(s_tm[1], qd1, kv_tile(sh, kst));
-      mma_commit(smem_u32(sh.bars + kBarSFull + 1));
+      issue_s<kFp8>(s_tm[1], qd1, kv_tile<kRopeQ>(sh, kst));
+      mma_commit(smem_u32(sh.bars + L::kSFull + 1));
     }
-    mma_commit(smem_u32(sh.bars + kBarKVEmpty + kst));
-    if (n == 1) mma_commit(smem_u32(sh.bars + kBarQEmpty));
+    mma_commit(smem_u32(sh.bars + L::kKVEmpty + kst));
+    if (n == 1) mma_commit(smem_u32(sh.bars + L::kQEmpty + qbuf));
     for (int j = 0; j < n; ++j) {
-      const int vst = kv_it % kStages;
-      if (!wait_bar(sh, p, kBarKVFull + vst, (kv_it / kStages) & 1, 12)) { ok = false; break; }
+      const int vst = kv_it % L::kStages;
+      if (!wait_bar(sh, p, L::kKVFull + vst, (kv_it / L::kStages) & 1, 12)) { ok = false; break; }
       ++kv_it;
       const bool more = j + 1 < n;
       if (more) {
-        kst = kv_it % kStages;
-        if (!wait_bar(sh, p, kBarKVFull + kst, (kv_it / kStages) & 1, 13)) { ok = false; break; }
+        kst = kv_it % L::kStages;
+        if (!wait_bar(sh, p, L::kKVFull + kst, (kv_it / L::kStages) & 1, 13)) { ok = false; break; }
         ++kv_it;
       }
       // tile 0
-      if (!wait_bar(sh, p, kBarPFull + 0, p_cnt[0] & 1, 14)) { ok = false; break; }
+      if (!wait_bar(sh, p, L::kPFull + 0, p_cnt[0] & 1, 14)) { ok = false; break; }
       ++p_cnt[0];
       tc_fence_after();
-      issue_pv(o_tm[0], s_tm[0], kv_tile(sh, vst), j > 0);
+      issue_pv(o_tm[0], s_tm[0], kv_tile<kRopeQ>(sh, vst), j > 0);
       if (more) {
-        issue_s<kFp8>(s_tm[0], qd0, kv_tile(sh, kst));
-        mma_commit(smem_u32(sh.bars + kBarSFull + 0));
+        issue_s<kFp8>(s_tm[0], qd0, kv_tile<kRopeQ>(sh, kst));
+        mma_commit(smem_u32(sh.bars + L::kSFull + 0));
       } else {
-        mma_commit(smem_u32(sh.bars + kBarOFull + 0));
+        mma_commit(smem_u32(sh.bars + L::kOFull + 0));
       }
       // tile 1
       if (live1) {
-        if (!wait_bar(sh, p, kBarPFull + 1, p_cnt[1] & 1, 15)) { ok = false; break; }
+        if (!wait_bar(sh, p, L::kPFull + 1, p_cnt[1] & 1, 15)) { ok = false; break; }
         ++p_cnt[1];
         tc_fence_after();
-        issue_pv(o_tm[1], s_tm[1], kv_tile(sh, vst), j > 0);
+        issue_pv(o_tm[1], s_tm[1], kv_tile<kRopeQ>(sh, vst), j > 0);
         if (more) {
-          issue_s<kFp8>(s_tm[1], qd1, kv_tile(sh, kst));
-          mma_commit(smem_u32(sh.bars + kBarSFull + 1));
+          issue_s<kFp8>(s_tm[1], qd1, kv_tile<kRopeQ>(sh, kst));
+          mma_commit(smem_u32(sh.bars + L::kSFull + 1));
         } else {
-          mma_commit(smem_u32(sh.bars + kBarOFull + 1));
+          mma_commit(smem_u32(sh.bars + L::kOFull + 1));
         }
       }
-      mma_commit(smem_u32(sh.bars + kBarKVEmpty + vst));
-      if (more) mma_commit(smem_u32(sh.bars + kBarKVEmpty + kst));
-      if (j + 2 == n) mma_commit(smem_u32(sh.bars + kBarQEmpty));
+      mma_commit(smem_u32(sh.bars + L::kKVEmpty + vst));
+      if (more) mma_commit(smem_u32(sh.bars + L::kKVEmpty + kst));
+      if (j + 2 == n) mma_commit(smem_u32(sh.bars + L::kQEmpty + qbuf));
     }
   }
   // all issued MMAs complete before TMEM is released
-  mma_commit(smem_u32(sh.bars + kBarMmaDone));
-  const uint32_t addr = smem_u32(sh.bars + kBarMmaDone);
+  mma_commit(smem_u32(sh.bars + L::kMmaDone));
+  const uint32_t addr = smem_u32(sh.bars + L::kMmaDone);
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(addr, 0) && global_timer_ns() - t0 < p.timeout_ns) {
   }
 }
 
-template <bool kFp8>
+// Softmax variants under measurement (0 = off).
+#ifndef WF_SPLIT_LD
+#define WF_SPLIT_LD 0
+#endif
+#ifndef WF_WARP_ARRIVE
+#define WF_WARP_ARRIVE 0
+#endif
+#ifndef WF_WIDE_MAX
+#define WF_WIDE_MAX 0
+#endif
+#ifndef WF_LANE0_WAIT
+#define WF_LANE0_WAIT 0
+#endif
+
+// exp2 of one row's 128 scores (scaled by sl2, minus the reference max m_ref)
+// stored as bf16 pairs into TMEM at s_tm; returns the row sum of the fp32
+// values.  Every exp2 runs on MUFU (masked columns hold -inf and give +0).
+// Moving a share of them to an FMA-pipe polynomial (a cubic on the fraction
+// plus an exponent add) measured slower at every share tried: 1/8, 1/4 and
+// 3/8 of the pairs gave 1058, 1052 and 1003 against 1124 TFLOP/s.  Four
+// independent partial sums keep the row sum off one serial chain.
+__device__ __forceinline__ float exp_to_p(const float (&s)[128], float sl2, float m_ref, uint32_t s_tm) {
+  const float2 sl2x2 = make_float2(sl2, sl2);
+  const float2 negm2 = make_float2(-m_ref, -m_ref);
+  float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const int pi = 16 * q4 + x;
+      const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
+      const float2 pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
+      ls[x & 3] = __fadd2_rn(ls[x & 3], pr);
+      pk[x] = pack_bf16x2(pr.x, pr.y);
+    }
+    tmem_st16(s_tm + 16 * q4, pk);
+  }
+  const float2 l01 = __fadd2_rn(ls[0], ls[1]), l23 = __fadd2_rn(ls[2], ls[3]);
+  const float2 lt = __fadd2_rn(l01, l23);
+  return lt.x + lt.y;
+}
+
+template <bool kFp8, bool kRopeQ>
 __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, uint32_t tmem, int t, int u0, int u1) {
+  using L = Layout<kRopeQ>;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int row_in_tile = (warp % 4) * 32 + lane;
@@ -463,10 +639,64 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
       } else {
         key_tile(c, j, tok, valid);
       }
-      if (!wait_bar(sh, p, kBarSFull + t, s_cnt & 1, 20 + t)) return;
+      // warp-uniform: the TMEM loads and stores below are warp-collective
+#if WF_LANE0_WAIT
+      {
+        // one lane polls the barrier; the warp synchronises on its result
+        bool okw = true;
+        if (lane == 0) okw = wait_bar(sh, p, L::kSFull + t, s_cnt & 1, 20 + t);
+        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, okw, 0)) return;
+      }
+#else
+      if (!__all_sync(0xffffffffu, wait_bar(sh, p, L::kSFull + t, s_cnt & 1, 20 + t))) return;
+#endif
       ++s_cnt;
       tc_fence_after();
       float s[128];
+      float mxs[8];
+#if WF_SPLIT_LD
+      // two halves: the second half's TMEM load is in flight while the
+      // first half's columns are reduced
+#pragma unroll
+      for (int q4 = 0; q4 < 2; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(s_tm + 32 * q4, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s[32 * q4 + x] = __uint_as_float(r[x]);
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int q4 = 2; q4 < 4; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(s_tm + 32 * q4, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s[32 * q4 + x] = __uint_as_float(r[x]);
+      }
+      if (valid < 64) {
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x >= valid) s[x] = -INFINITY;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(s[c], s[c + 8]);
+#pragma unroll
+      for (int x = 16; x < 64; x += 16) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
+      }
+      tmem_wait_ld();
+      if (valid < 128) {
+#pragma unroll
+        for (int x = 64; x < 128; ++x)
+          if (x >= valid) s[x] = -INFINITY;
+      }
+#pragma unroll
+      for (int x = 64; x < 128; x += 16) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
+      }
+#else
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t r[32];
@@ -480,7 +710,17 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
         for (int x = 0; x < 128; ++x)
           if (x >= valid) s[x] = -INFINITY;
       }
-      float mxs[8];
+#if WF_WIDE_MAX
+      // a shallower reduction: 32 three-input maxima over disjoint quadruples
+      // (depth 2), then a tree (depth 4) -- 6 dependent steps instead of 11
+      {
+        float m32[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) m32[c] = max3f(s[4 * c], s[4 * c + 1], fmaxf(s[4 * c + 2], s[4 * c + 3]));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(max3f(m32[c], m32[c + 8], m32[c + 16]), m32[c + 24]);
+      }
+#else
 #pragma unroll
       for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(s[c], s[c + 8]);
 #pragma unroll
@@ -488,6 +728,8 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
 #pragma unroll
         for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
       }
+#endif
+#endif
       const float mx = fmaxf(max3f(mxs[0], mxs[1], mxs[2]), max3f(mxs[3], max3f(mxs[4], mxs[5], mxs[6]), mxs[7]));
       const float m_new = fmaxf(m_ref, mx * sl2);
       if (j == t0) {
@@ -512,35 +754,22 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
           }
         }
       }
-      // exp2 on MUFU for every score (an FMA-pipe polynomial for part of them
-      // measured slower here); four independent partial sums keep the row sum
-      // off one serial chain of adds.  Masked columns hold -inf: ex2 gives +0.
-      const float2 sl2x2 = make_float2(sl2, sl2);
-      const float2 negm2 = make_float2(-m_ref, -m_ref);
-      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int pi = 16 * q4 + x;
-          const float2 v = __ffma2_rn(make_float2(s[2 * pi], s[2 * pi + 1]), sl2x2, negm2);
-          const float2 pr = make_float2(fast_exp2(v.x), fast_exp2(v.y));
-          ls[x & 3] = __fadd2_rn(ls[x & 3], pr);
-          pk[x] = pack_bf16x2(pr.x, pr.y);
-        }
-        tmem_st16(s_tm + 16 * q4, pk);
-      }
-      const float2 l01 = __fadd2_rn(ls[0], ls[1]), l23 = __fadd2_rn(ls[2], ls[3]);
-      const float2 lt = __fadd2_rn(l01, l23);
-      l += lt.x + lt.y;
+      // P = exp2(s * sl2 - m_ref) into TMEM over S's first 64 columns
+      l += exp_to_p(s, sl2, m_ref, s_tm);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(sh.bars + kBarPFull + t));
+#if WF_WARP_ARRIVE
+      // one arrival per warp (after every lane's stores have completed): 128
+      // per-thread arrivals on one barrier took ~250 cycles to land
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(sh.bars + L::kPFull + t));
+#else
+      mbar_arrive(smem_u32(sh.bars + L::kPFull + t));
+#endif
     }
     // epilogue: O / l -> bf16 rows of this tile (a part of a split unit:
     // fp32 rows and the LSE into its partial slot, merged by the combine pass)
-    if (!wait_bar(sh, p, kBarOFull + t, o_cnt & 1, 24 + t)) return;
+    if (!__all_sync(0xffffffffu, wait_bar(sh, p, L::kOFull + t, o_cnt & 1, 24 + t))) return;
     ++o_cnt;
     tc_fence_after();
     const float inv_l = 1.0f / l;
@@ -587,22 +816,37 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
   }
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kRopeQ>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using L = Layout<kRopeQ>;
   extern __shared__ uint8_t smem_raw[];
-  const Shared sh = carve_smem(smem_raw);
+  const Shared sh = carve_smem<kRopeQ>(smem_raw);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
   if (warp == 9 && lane == 0) {
-    for (int b = 0; b < kNumBars; ++b) {
+    for (int b = 0; b < L::kNumBars; ++b) {
       uint32_t count = 1;
-      if (b == kBarPFull || b == kBarPFull + 1) count = 128;
+      if (b == L::kPFull || b == L::kPFull + 1) count = WF_WARP_ARRIVE ? 4 : 128;  // the tile's softmax warps
+      if (kRopeQ && b >= L::kQFull && b < L::kQFull + L::kQBufs) count = WF_WARP_ARRIVE ? 2 : 64;  // rotation
       mbar_init(smem_u32(sh.bars + b), count);
     }
     *sh.abort_flag = 0;
+    if (kRopeQ) {
+      RopeConsts rc;
+      rc.fw = uint32_t(p.plan->fw);
+      rc.fhw = uint32_t(p.plan->fh) * rc.fw;
+      rc.F = uint32_t(p.plan->F);
+      rc.Pt = p.plan->Pt;
+      rc.Ph = p.plan->Ph;
+      rc.Pw = p.plan->Pw;
+      rc.off_t = uint32_t(p.plan->off_rope_t);
+      rc.off_h = uint32_t(p.plan->off_rope_h);
+      rc.off_w = uint32_t(p.plan->off_rope_w);
+      *sh.rope = rc;
+    }
     fence_barrier_init();
     fence_proxy_async_smem();
     tma_prefetch_desc(&tm_q);
@@ -622,14 +866,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role<kFp8>(sh, p, tmem, warp / 4, u0, u1);
+    softmax_role<kFp8, kRopeQ>(sh, p, tmem, warp / 4, u0, u1);
   } else {
     regs_decrease<kControlRegs>();
     if (warp == 8) {
-      if (lane == 0) mma_issuer<kFp8>(sh, p, tmem, u0, u1);
+      if (lane == 0) mma_issuer<kFp8, kRopeQ>(sh, p, tmem, u0, u1);
       __syncwarp();
-    } else if (warp == 9 && lane == 0) {
-      producer<kFp8>(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
+    } else if (warp == 9) {
+      if (lane == 0) producer<kFp8, kRopeQ>(sh, p, &tm_q, &tm_k, &tm_v, u0, u1);
+    } else if (kRopeQ) {
+      rope_q_role(sh, p, u0, u1);
     }
   }
   tc_fence_before();
@@ -685,16 +931,17 @@ bool make_tmap(CUtensorMap* tm, const void* base, int64_t tokens, int32_t H, boo
   return r == CUDA_SUCCESS ? true : report("cuTensorMapEncodeTiled", int(r));
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kRopeQ>
 wf_status launch(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q, const float* q_scales,
                  const void* k_pool, const float* k_scales, const void* v_pool, void* out, float* lse, float scale,
                  void* workspace, uint64_t timeout_ns, cudaStream_t stream) {
   static int attr_done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WF_ERR_CUDA;
-  if (dev < 64 && !attr_done[dev]) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(attn_fwd_sm100<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (dev < 0 || dev >= 64) return WF_ERR_UNSUPPORTED;
+  if (!attr_done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100<kFp8, kRopeQ>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<kRopeQ>::kSmemBytes);
     if (e != cudaSuccess) {
       report(cudaGetErrorString(e), int(e));
       cudaGetLastError();
@@ -728,12 +975,13 @@ wf_status launch(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q, c
   // partial slots after the status block (used only by split units)
   p.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + WF_ATTN_STATUS_BYTES);
   p.part_lse = p.part_o + int64_t(h->num_units) * 256 * 128;
-  attn_fwd_sm100<kFp8><<<h->num_ctas, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+  p.plan = reinterpret_cast<const wf_plan_hdr*>(dev_plan);
+  attn_fwd_sm100<kFp8, kRopeQ><<<h->num_ctas, kThreads, Layout<kRopeQ>::kSmemBytes, stream>>>(tq, tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     report(cudaGetErrorString(e), int(e));
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_sm100<kFp8>) == cudaSuccess) {
+    if (cudaFuncGetAttributes(&fa, attn_fwd_sm100<kFp8, kRopeQ>) == cudaSuccess) {
       char msg[256];
       std::snprintf(msg, sizeof(msg), "attributes: regs %d, max threads %d, static smem %zu, max dyn smem %d",
                     fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes, fa.maxDynamicSharedSizeBytes);
@@ -750,16 +998,24 @@ wf_status launch(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q, c
 wf_status launch_attn_sm100(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_rot, const void* k_pool,
                             const void* v_pool, void* out, float* lse, float scale, void* workspace,
                             uint64_t timeout_ns, cudaStream_t stream) {
-  return launch<false>(h, dev_plan, q_rot, nullptr, k_pool, nullptr, v_pool, out, lse, scale, workspace, timeout_ns,
-                       stream);
+  return launch<false, false>(h, dev_plan, q_rot, nullptr, k_pool, nullptr, v_pool, out, lse, scale, workspace,
+                              timeout_ns, stream);
+}
+
+// The same from the raw (not yet rotated) queries: the kernel applies Q's RoPE.
+wf_status launch_attn_sm100_rope_q(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q_raw,
+                                   const void* k_pool, const void* v_pool, void* out, float* lse, float scale,
+                                   void* workspace, uint64_t timeout_ns, cudaStream_t stream) {
+  return launch<false, true>(h, dev_plan, q_raw, nullptr, k_pool, nullptr, v_pool, out, lse, scale, workspace,
+                             timeout_ns, stream);
 }
 
 // The same with e4m3 Q and K codes and their block scales.
 wf_status launch_attn_sm100_fp8(const wf_plan_hdr* h, const uint8_t* dev_plan, const void* q8, const float* q_scales,
                                 const void* k8_pool, const float* k_scales, const void* v_pool, void* out, float* lse,
                                 float scale, void* workspace, uint64_t timeout_ns, cudaStream_t stream) {
-  return launch<true>(h, dev_plan, q8, q_scales, k8_pool, k_scales, v_pool, out, lse, scale, workspace, timeout_ns,
-                      stream);
+  return launch<true, false>(h, dev_plan, q8, q_scales, k8_pool, k_scales, v_pool, out, lse, scale, workspace,
+                             timeout_ns, stream);
 }
 
 }  // namespace wf

@@ -1,25 +1,23 @@
 // wf_rope3d_append: 3D rotary embedding of the round's new Q and K, fused
-// with the append of K'/V into the ring pool.
+// with the append of K'/V into the ring pool (and wf_rope3d_append_kv, the
+// same without the queries).
 //
-// HBM-bound: per (token, head) row it reads Q, K, V and writes Q', K', V
-// (6 * D * elem bytes).  Each thread moves one 16-byte vector of each
+// HBM-bound in bytes, but the bit-exact fp64 rotation makes it instruction-
+// and conversion-heavy: per (token, head) row it reads Q, K, V and writes Q',
+// K', V (6 * D * elem bytes).  Each thread moves one 16-byte vector of each
 // tensor; a warp covers consecutive vectors, so every load and store is a
-// fully coalesced 512-byte run.  (Two vectors per thread, all six loads in
-// flight, needed 74 registers and measured 3% slower than one vector at 60
-// registers with four blocks per SM.)  Index decoding uses exact multiply-shift
-// reciprocals instead of integer division.  The rotation runs in fp64 from the plan's fp64
-// cos/sin tables (L1-resident, a few KB) and is rounded once to the storage
-// type: fp64 -> fp32 with round-to-odd, then fp32 -> bf16 to nearest even,
-// which equals direct nearest-even rounding of the fp64 value (Boldo and
-// Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms
-// using rounding to odd", IEEE TC 2008: rounding to odd in a format with at
-// least two more bits makes the second rounding correct).
+// fully coalesced 512-byte run.  Index decoding uses exact multiply-shift
+// reciprocals instead of integer division.  The rotation runs in fp64 from
+// the plan's fp64 cos/sin tables (L1-resident, a few KB) and is rounded once
+// to the storage type (rope_math.cuh).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "wf.h"
+#include "rope_math.cuh"
 #include "wf_plan.h"
 
 namespace {
@@ -56,63 +54,9 @@ struct RopeParams {
   int64_t nvec;          // vectors in the new tensors
 };
 
-__device__ __forceinline__ float f64_to_f32_round_odd(double x) {
-  float r = __double2float_rz(x);
-  if (double(r) != x) r = __int_as_float(__float_as_int(r) | 1);
-  return r;
-}
-
-__device__ __forceinline__ void rotate_pair(double x, double y, double2 cs, double& xr, double& yr) {
-  // same operation order as a plain fp64 evaluation of x*c - y*s, x*s + y*c
-  xr = __dsub_rn(__dmul_rn(x, cs.x), __dmul_rn(y, cs.y));
-  yr = __dadd_rn(__dmul_rn(x, cs.y), __dmul_rn(y, cs.x));
-}
-
-template <typename T>
-struct Pack;
-
-template <>
-struct Pack<__nv_bfloat16> {
-  static constexpr int kElems = 8;
-  __device__ static void unpack(const uint4& v, double* out) {
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 f = __bfloat1622float2(p[i]);
-      out[2 * i] = f.x;
-      out[2 * i + 1] = f.y;
-    }
-  }
-  __device__ static uint4 pack(const double* in) {
-    uint4 v;
-    __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      p[i] = __floats2bfloat162_rn(f64_to_f32_round_odd(in[2 * i]), f64_to_f32_round_odd(in[2 * i + 1]));
-    return v;
-  }
-};
-
-template <>
-struct Pack<float> {
-  static constexpr int kElems = 4;
-  __device__ static void unpack(const uint4& v, double* out) {
-    const float* p = reinterpret_cast<const float*>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) out[i] = p[i];
-  }
-  __device__ static uint4 pack(const double* in) {
-    uint4 v;
-    float* p = reinterpret_cast<float*>(&v);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = __double2float_rn(in[i]);
-    return v;
-  }
-};
-
-// Rotate and store one 16-byte vector of Q and K (and copy V) given its flat
-// index e in the [R*C, H, D] tensors.
-template <typename T>
+// Rotate and store one 16-byte vector of Q (kWithQ) and K, and copy V, given
+// its flat index e in the [R*C, H, D] tensors.
+template <typename T, bool kWithQ>
 __device__ __forceinline__ void rope_vector(const RopeParams& p, uint32_t e, const uint4& qv, const uint4& kv,
                                             const uint4& vv, uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
                                             uint4* __restrict__ v_pool) {
@@ -128,51 +72,52 @@ __device__ __forceinline__ void rope_vector(const RopeParams& p, uint32_t e, con
   const uint32_t hh = fdiv(l, p.div_fw);
   const uint32_t ww = l - hh * uint32_t(p.fw);
   double qd[E], kd[E];
-  Pack<T>::unpack(qv, qd);
+  if (kWithQ) Pack<T>::unpack(qv, qd);
   Pack<T>::unpack(kv, kd);
 #pragma unroll
   for (int u = 0; u < E / 2; ++u) {
     const int32_t m = int32_t(vin) * (E / 2) + u;  // pair index in [0, D/2)
-    double2 cs;
-    if (m < p.Pt) {
-      cs = __ldg(p.tab_t + int64_t(i * p.F + f) * p.Pt + m);
-    } else if (m < p.Pt + p.Ph) {
-      cs = __ldg(p.tab_h + int64_t(hh) * p.Ph + (m - p.Pt));
-    } else {
-      cs = __ldg(p.tab_w + int64_t(ww) * p.Pw + (m - p.Pt - p.Ph));
-    }
-    rotate_pair(qd[2 * u], qd[2 * u + 1], cs, qd[2 * u], qd[2 * u + 1]);
+    const double2 cs = rope_cos_sin(p.tab_t, p.tab_h, p.tab_w, p.Pt, p.Ph, p.Pw, i * p.F + f, hh, ww, m);
+    if (kWithQ) rotate_pair(qd[2 * u], qd[2 * u + 1], cs, qd[2 * u], qd[2 * u + 1]);
     rotate_pair(kd[2 * u], kd[2 * u + 1], cs, kd[2 * u], kd[2 * u + 1]);
   }
   const int64_t dst = ((int64_t(p.slot[i]) * p.C + j) * p.H + head) * p.div_vpr.d + vin;
-  __stcs(q_rot + e, Pack<T>::pack(qd));
+  if (kWithQ) __stcs(q_rot + e, Pack<T>::pack(qd));
   __stcs(k_pool + dst, Pack<T>::pack(kd));
   __stcs(v_pool + dst, vv);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) rope3d_append_kernel(RopeParams p, const uint4* __restrict__ q,
-                                                            const uint4* __restrict__ k,
-                                                            const uint4* __restrict__ v,
-                                                            uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
-                                                            uint4* __restrict__ v_pool) {
-  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+constexpr int kRopeThreads = 256;
+
+// One 16-byte vector of each tensor per thread, a block per 256 vectors
+// (61 registers: four blocks per SM).  Measured slower on the 4-chunk round (72 us
+// for this kernel): a grid-stride loop that keeps 3-5 further steps' loads in
+// flight through cp.async into shared memory (85-98 us), half vectors per
+// thread at 6 or 8 blocks per SM (82 us, issue-bound at 75% issue activity),
+// and converting bf16 -> fp64 or testing the round-to-odd exactness with
+// integer operations instead of conversions (83-91 us).
+template <typename T, bool kWithQ>
+__global__ void __launch_bounds__(kRopeThreads)
+    rope3d_append_kernel(RopeParams p, const uint4* __restrict__ q, const uint4* __restrict__ k,
+                         const uint4* __restrict__ v, uint4* __restrict__ q_rot, uint4* __restrict__ k_pool,
+                         uint4* __restrict__ v_pool) {
+  const int64_t e = int64_t(blockIdx.x) * kRopeThreads + threadIdx.x;
   if (e >= p.nvec) return;
-  const uint4 qv = __ldcs(q + e), kv = __ldcs(k + e), vv = __ldcs(v + e);
-  rope_vector<T>(p, uint32_t(e), qv, kv, vv, q_rot, k_pool, v_pool);
+  const uint4 qv = kWithQ ? __ldcs(q + e) : make_uint4(0, 0, 0, 0);
+  const uint4 kv = __ldcs(k + e), vv = __ldcs(v + e);
+  rope_vector<T, kWithQ>(p, uint32_t(e), qv, kv, vv, q_rot, k_pool, v_pool);
 }
 
 bool misaligned(const void* ptr) { return reinterpret_cast<uintptr_t>(ptr) % 16 != 0; }
 
-}  // namespace
 
-extern "C" wf_status wf_rope3d_append(const void* host_plan, const void* dev_plan, const void* q, const void* k,
-                                      const void* v, void* q_rot, void* k_pool, void* v_pool,
-                                      wf_stream_t stream) {
-  if (!host_plan || !dev_plan || !q || !k || !v || !q_rot || !k_pool || !v_pool) return WF_ERR_INVALID_ARG;
+// Shared by the two entry points; q / q_rot are null for the K/V-only append.
+wf_status rope_append(const void* host_plan, const void* dev_plan, const void* q, const void* k, const void* v,
+                      void* q_rot, void* k_pool, void* v_pool, wf_stream_t stream) {
+  const bool with_q = q != nullptr;
   const wf_plan_hdr* h = static_cast<const wf_plan_hdr*>(host_plan);
   if (h->magic != WF_PLAN_MAGIC || h->version != WF_PLAN_VERSION) return WF_ERR_PLAN;
-  if (misaligned(dev_plan) || misaligned(q) || misaligned(k) || misaligned(v) || misaligned(q_rot) ||
+  if (misaligned(dev_plan) || (with_q && (misaligned(q) || misaligned(q_rot))) || misaligned(k) || misaligned(v) ||
       misaligned(k_pool) || misaligned(v_pool))
     return WF_ERR_ALIGNMENT;
   const int elem = h->dtype == WF_BF16 ? 2 : 4;
@@ -196,9 +141,9 @@ extern "C" wf_status wf_rope3d_append(const void* host_plan, const void* dev_pla
   p.div_fhw = make_fastdiv(uint32_t(h->fh * h->fw));
   p.div_fw = make_fastdiv(uint32_t(h->fw));
 
-  const int threads = 256;
-  const int64_t blocks = (p.nvec + threads - 1) / threads;
-  if (blocks > 0x7FFFFFFF) return WF_ERR_CAPACITY;
+  const int64_t nblocks = (p.nvec + kRopeThreads - 1) / kRopeThreads;
+  if (nblocks > 0x7FFFFFFF) return WF_ERR_CAPACITY;
+  const unsigned blocks = unsigned(nblocks);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint4* q4 = static_cast<const uint4*>(q);
   const uint4* k4 = static_cast<const uint4*>(k);
@@ -206,10 +151,30 @@ extern "C" wf_status wf_rope3d_append(const void* host_plan, const void* dev_pla
   uint4* qr4 = static_cast<uint4*>(q_rot);
   uint4* kp4 = static_cast<uint4*>(k_pool);
   uint4* vp4 = static_cast<uint4*>(v_pool);
-  if (h->dtype == WF_BF16)
-    rope3d_append_kernel<__nv_bfloat16><<<unsigned(blocks), threads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
+  const bool bf16 = h->dtype == WF_BF16;
+  if (with_q && bf16)
+    rope3d_append_kernel<__nv_bfloat16, true><<<blocks, kRopeThreads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
+  else if (with_q)
+    rope3d_append_kernel<float, true><<<blocks, kRopeThreads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
+  else if (bf16)
+    rope3d_append_kernel<__nv_bfloat16, false><<<blocks, kRopeThreads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
   else
-    rope3d_append_kernel<float><<<unsigned(blocks), threads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
+    rope3d_append_kernel<float, false><<<blocks, kRopeThreads, 0, s>>>(p, q4, k4, v4, qr4, kp4, vp4);
   if (cudaGetLastError() != cudaSuccess) return WF_ERR_CUDA;
   return WF_OK;
+}
+
+}  // namespace
+
+extern "C" wf_status wf_rope3d_append(const void* host_plan, const void* dev_plan, const void* q, const void* k,
+                                      const void* v, void* q_rot, void* k_pool, void* v_pool,
+                                      wf_stream_t stream) {
+  if (!host_plan || !dev_plan || !q || !k || !v || !q_rot || !k_pool || !v_pool) return WF_ERR_INVALID_ARG;
+  return rope_append(host_plan, dev_plan, q, k, v, q_rot, k_pool, v_pool, stream);
+}
+
+extern "C" wf_status wf_rope3d_append_kv(const void* host_plan, const void* dev_plan, const void* k, const void* v,
+                                         void* k_pool, void* v_pool, wf_stream_t stream) {
+  if (!host_plan || !dev_plan || !k || !v || !k_pool || !v_pool) return WF_ERR_INVALID_ARG;
+  return rope_append(host_plan, dev_plan, nullptr, k, v, nullptr, k_pool, v_pool, stream);
 }

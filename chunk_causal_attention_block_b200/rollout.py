@@ -97,7 +97,7 @@ class Rollout:
 
     def __init__(self, cfg: RoundConfig, device="cuda", seed: int = 42, first_n0: Optional[int] = None,
                  num_ctas: int = 0, want_lse: bool = True, stream: Optional[torch.cuda.Stream] = None,
-                 fp8: bool = False):
+                 fp8: bool = False, fused_q_rope: bool = False):
         self.cfg = cfg
         self.device = torch.device(device)
         self.seed = seed
@@ -116,6 +116,11 @@ class Rollout:
         self.q_rot = torch.empty(nq, H, D, **kw)
         self.out = torch.empty(nq, H, D, **kw)
         self.lse = torch.empty(H, nq, dtype=torch.float32, device=self.device) if want_lse else None
+        # fused_q_rope: the attention rotates the raw Q itself (wf_chunk_causal_attn_rope)
+        # and the append writes only K'/V (wf_rope3d_append_kv)
+        if fused_q_rope and (fp8 or cfg.dtype != wf.WF_BF16):
+            raise ValueError("the fused Q-RoPE path takes bf16 rounds with 16-bit scores")
+        self.fused_q_rope = fused_q_rope
         # 8-bit scores: e4m3 codes of Q' and of the pool's K' with their block scales
         self.fp8 = fp8
         if fp8:
@@ -185,8 +190,8 @@ class Rollout:
             g = min(c.R, self.first_n0 - n)
             self.fill_inputs(n, g, -1)
             self._plan(self.desc(n, R=g, Wc=0, noise=[0] * g))
-            wf.wf_rope3d_append(self.host_plan, self.dev_plan, self.q, self.k, self.v, self.q_rot, self.k_pool,
-                                self.v_pool, self.stream)
+            wf.wf_rope3d_append_kv(self.host_plan, self.dev_plan, self.k, self.v, self.k_pool, self.v_pool,
+                                   self.stream)
             if self.fp8:
                 wf.wf_quantize_fp8(self.host_plan, self.k_pool, self.k8_pool, self.k_scales, wf.WF_FP8_K, self.stream)
             n += g
@@ -200,6 +205,10 @@ class Rollout:
         self._plan(self.desc(self.n0_of(r)))
 
     def append(self):
+        if self.fused_q_rope:
+            wf.wf_rope3d_append_kv(self.host_plan, self.dev_plan, self.k, self.v, self.k_pool, self.v_pool,
+                                   self.stream)
+            return
         wf.wf_rope3d_append(self.host_plan, self.dev_plan, self.q, self.k, self.v, self.q_rot, self.k_pool,
                             self.v_pool, self.stream)
         if self.fp8:
@@ -215,6 +224,9 @@ class Rollout:
             wf.wf_chunk_causal_attn_fp8(self.host_plan, self.dev_plan, self.q8, self.q_scales, self.k8_pool,
                                         self.k_scales, self.v_pool, self.out, self.lse, scale, self.workspace,
                                         self.stream)
+        elif self.fused_q_rope:
+            wf.wf_chunk_causal_attn_rope(self.host_plan, self.dev_plan, self.q, self.k_pool, self.v_pool, self.out,
+                                         self.lse, scale, self.workspace, self.stream)
         else:
             wf.wf_chunk_causal_attn(self.host_plan, self.dev_plan, self.q_rot, self.k_pool, self.v_pool, self.out,
                                     self.lse, scale, self.workspace, self.stream)

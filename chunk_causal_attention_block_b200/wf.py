@@ -30,7 +30,8 @@ WF_FP8_Q, WF_FP8_K = 0, 1
 
 # exported symbols, in the order include/wf.h and include/wf_synth.h declare them
 EXPORTS = ("wf_plan_bytes", "wf_plan_round", "wf_balance_units", "wf_rope3d_append", "wf_attn_workspace_bytes",
-           "wf_attn_workspace_init", "wf_attn_workspace_status", "wf_chunk_causal_attn",
+           "wf_attn_workspace_init", "wf_attn_workspace_status", "wf_chunk_causal_attn", "wf_rope3d_append_kv",
+           "wf_chunk_causal_attn_rope",
            "wf_chunk_causal_attn_noalloc", "wf_quantize_fp8", "wf_chunk_causal_attn_fp8", "wf_status_string",
            "wf_version", "wf_synth_fill")
 
@@ -83,6 +84,9 @@ def lib() -> ctypes.CDLL:
         L.wf_plan_round.argtypes, L.wf_plan_round.restype = [dp, vp, sz, vp, sz, vp], i32
         L.wf_balance_units.argtypes, L.wf_balance_units.restype = [vp, i32, i32, vp, vp], i32
         L.wf_rope3d_append.argtypes, L.wf_rope3d_append.restype = [vp] * 8 + [vp], i32
+        L.wf_rope3d_append_kv.argtypes, L.wf_rope3d_append_kv.restype = [vp] * 6 + [vp], i32
+        L.wf_chunk_causal_attn_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp]
+        L.wf_chunk_causal_attn_rope.restype = i32
         L.wf_attn_workspace_bytes.argtypes, L.wf_attn_workspace_bytes.restype = [vp], sz
         L.wf_attn_workspace_init.argtypes, L.wf_attn_workspace_init.restype = [vp, sz, vp], i32
         L.wf_attn_workspace_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -162,6 +166,11 @@ def wf_rope3d_append(host_plan, dev_plan, q, k, v, q_rot, k_pool, v_pool, stream
                                   _ptr(k_pool), _ptr(v_pool), _stream(stream)), "wf_rope3d_append")
 
 
+def wf_rope3d_append_kv(host_plan, dev_plan, k, v, k_pool, v_pool, stream=None):
+    _check(lib().wf_rope3d_append_kv(_ptr(host_plan), _ptr(dev_plan), _ptr(k), _ptr(v), _ptr(k_pool), _ptr(v_pool),
+                                     _stream(stream)), "wf_rope3d_append_kv")
+
+
 def wf_attn_workspace_bytes(host_plan) -> int:
     return lib().wf_attn_workspace_bytes(_ptr(host_plan))
 
@@ -184,6 +193,15 @@ def wf_chunk_causal_attn(host_plan, dev_plan, q_rot, k_pool, v_pool, out, lse=No
     _check(lib().wf_chunk_causal_attn(_ptr(host_plan), _ptr(dev_plan), _ptr(q_rot), _ptr(k_pool), _ptr(v_pool),
                                       _ptr(out), _ptr(lse), float(softmax_scale), _ptr(workspace), wb,
                                       _stream(stream)), "wf_chunk_causal_attn")
+
+
+def wf_chunk_causal_attn_rope(host_plan, dev_plan, q, k_pool, v_pool, out, lse=None, softmax_scale=0.0,
+                              workspace=None, stream=None, workspace_bytes=None):
+    """wf_chunk_causal_attn from raw queries: the kernel applies Q's RoPE."""
+    wb = workspace_bytes if workspace_bytes is not None else _nbytes(workspace)
+    _check(lib().wf_chunk_causal_attn_rope(_ptr(host_plan), _ptr(dev_plan), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                           _ptr(out), _ptr(lse), float(softmax_scale), _ptr(workspace), wb,
+                                           _stream(stream)), "wf_chunk_causal_attn_rope")
 
 
 def wf_chunk_causal_attn_noalloc(host_plan, dev_plan, q_rot, k_pool, v_pool, out, lse=None, softmax_scale=0.0,

@@ -181,6 +181,15 @@ wf_status wf_rope3d_append(const void* host_plan, const void* dev_plan,
                            const void* q, const void* k, const void* v,
                            void* q_rot, void* k_pool, void* v_pool, wf_stream_t stream);
 
+/*
+ * wf_rope3d_append_kv -- wf_rope3d_append without the queries: rotates the
+ * new K and appends K'/V into the pool exactly as wf_rope3d_append does, and
+ * neither reads Q nor writes Q'.  Pair it with wf_chunk_causal_attn_rope,
+ * which rotates Q itself.  Arguments and errors as wf_rope3d_append.
+ */
+wf_status wf_rope3d_append_kv(const void* host_plan, const void* dev_plan, const void* k, const void* v,
+                              void* k_pool, void* v_pool, wf_stream_t stream);
+
 /* Bytes of attention workspace the plan's kernels need: the 256-byte status
  * block, plus 256 rows x (128 + 1) fp32 per unit when the plan splits units'
  * keys (see wf_plan_round); 0 for an invalid plan. */
@@ -214,6 +223,10 @@ wf_status wf_attn_workspace_status(const void* workspace, wf_stream_t stream, in
  *
  * q_rot:  device [R*C, H, D] (the output of wf_rope3d_append).
  * k_pool, v_pool: device [S*C, H, D] ring pool holding every visible chunk.
+ *         Every slot must hold finite values (zero a new pool once): the last
+ *         128-key tile of a visible run may extend into the next slot, whose
+ *         keys are masked out of the softmax (weight exactly 0) but still
+ *         enter the P*V product, where 0 * inf or 0 * NaN would be NaN.
  * out:    device [R*C, H, D] (written).
  * lse:    device fp32 [H, R*C] (natural-log sum of exp of scaled scores), or NULL.
  * softmax_scale: 0 means 1/sqrt(D).
@@ -229,6 +242,24 @@ wf_status wf_chunk_causal_attn(const void* host_plan, const void* dev_plan,
                                const void* q_rot, const void* k_pool, const void* v_pool,
                                void* out, float* lse, float softmax_scale,
                                void* workspace, size_t workspace_bytes, wf_stream_t stream);
+
+/*
+ * wf_chunk_causal_attn_rope -- wf_chunk_causal_attn from the round's raw
+ * (not yet rotated) queries: the attention kernel applies Q's 3D RoPE itself,
+ * on each unit's query tiles in shared memory, with the same fp64 rotation and
+ * single rounding to bf16 as wf_rope3d_append, so O and LSE are bit-identical
+ * to wf_rope3d_append followed by wf_chunk_causal_attn.  This saves writing
+ * and re-reading Q' (a third of the RoPE/append traffic) and the Q' buffer.
+ *
+ * q:      device [R*C, H, D] raw queries (read only).
+ * The pool must already hold this round's K'/V (wf_rope3d_append_kv).  All
+ * other arguments and the errors are those of wf_chunk_causal_attn; bf16
+ * plans with D = 128 only (else WF_ERR_UNSUPPORTED).
+ */
+wf_status wf_chunk_causal_attn_rope(const void* host_plan, const void* dev_plan, const void* q,
+                                    const void* k_pool, const void* v_pool, void* out, float* lse,
+                                    float softmax_scale, void* workspace, size_t workspace_bytes,
+                                    wf_stream_t stream);
 
 /*
  * wf_chunk_causal_attn_noalloc -- wf_chunk_causal_attn for callers that cannot
@@ -269,8 +300,10 @@ wf_status wf_chunk_causal_attn_noalloc(const void* host_plan, const void* dev_pl
  *
  * Blocks are WF_FP8_BLOCK consecutive tokens of one chunk (chunk-relative,
  * the last one ragged: nblk = ceil(C / WF_FP8_BLOCK) per chunk) times one
- * head.  scale = amax / 448 and inv = 448 / amax in fp32 (both 1 for an
- * all-zero block); each element becomes the e4m3 value nearest x * inv (one
+ * head.  scale = amax / 448 and inv = 448 / amax in fp32 (both 1 for a
+ * block whose 448 / amax is not finite: amax 0, or below 448 / FLT_MAX, about
+ * 1.3e-36, whose codes are then all zero); each element becomes the e4m3
+ * value nearest x * inv (one
  * fp32 product, then the nearest-even conversion that saturates at +-448),
  * and is read back as code * scale.
  */

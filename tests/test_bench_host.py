@@ -29,7 +29,8 @@ def test_kernel_hash_ignores_comments_and_blank_lines_but_not_code():
     assert bench.kernel_source_sha(_reader()) == base
     commented = _reader(lambda n, t: t.replace("\n", "\n\n// a note\n", 3) if n == "attn_sm100.cu" else t)
     assert bench.kernel_source_sha(commented) == base
-    changed = _reader(lambda n, t: t.replace("kStages = 4", "kStages = 5") if n == "attn_sm100.cu" else t)
+    changed = _reader(lambda n, t: t.replace("kStages = kRopeQ ? 3 : 4", "kStages = kRopeQ ? 3 : 5")
+                      if n == "attn_sm100.cu" else t)
     assert bench.kernel_source_sha(changed) != base
 
 

@@ -143,6 +143,30 @@ def test_fp8_entry_points_reject_bad_arguments_before_any_launch():
         assert e.value.code == code
 
 
+def test_fused_rope_entry_points_reject_bad_arguments_before_any_launch():
+    f32 = _plan(_desc())
+    bf16 = _plan(_desc(D=128, dtype=wf.WF_BF16))
+    fake = 1 << 20  # never dereferenced: validation fails first
+    cases = [
+        (lambda: wf.wf_rope3d_append_kv(bf16, fake, fake, None, fake, fake), wf.WF_ERR_INVALID_ARG),
+        (lambda: wf.wf_rope3d_append_kv(bf16, fake, fake, fake, fake + 4, fake), wf.WF_ERR_ALIGNMENT),
+        (lambda: wf.wf_chunk_causal_attn_rope(bf16, fake, fake, fake, fake, fake, None, 0.0, fake,
+                                              workspace_bytes=16), wf.WF_ERR_WORKSPACE),
+        (lambda: wf.wf_chunk_causal_attn_rope(bf16, fake, None, fake, fake, fake, None, 0.0, fake,
+                                              workspace_bytes=4096), wf.WF_ERR_INVALID_ARG),
+        (lambda: wf.wf_chunk_causal_attn_rope(bf16, fake, fake + 8, fake, fake, fake, None, 0.0, fake,
+                                              workspace_bytes=4096), wf.WF_ERR_ALIGNMENT),
+        (lambda: wf.wf_chunk_causal_attn_rope(f32, fake, fake, fake, fake, fake, None, 0.0, fake,
+                                              workspace_bytes=4096), wf.WF_ERR_UNSUPPORTED),
+        (lambda: wf.wf_chunk_causal_attn_rope(bf16, fake, fake, fake, fake, fake, None, -1.0, fake,
+                                              workspace_bytes=4096), wf.WF_ERR_INVALID_ARG),
+    ]
+    for call, code in cases:
+        with pytest.raises(wf.WfError) as e:
+            call()
+        assert e.value.code == code
+
+
 def test_workspace_size_follows_the_key_split():
     # one 1560-token chunk, 2 heads: 14 units for 148 CTAs -> each unit's keys in 4 parts
     d = wf.make_desc(2, 128, 30, 52, 1, 2, 1, 2, [1000], dtype=wf.WF_BF16, num_ctas=148)

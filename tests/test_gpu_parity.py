@@ -260,3 +260,42 @@ def test_fp32_and_bf16_paths_agree_on_wan_shaped_data():
     b.attend()
     torch.cuda.synchronize()
     gc.assert_bf16_close(gc.to_np(a.out), gc.to_np(b.out), "fp32 vs bf16 kernels")
+
+
+# ---------------------------------------------------------------- Q's RoPE inside the attention
+
+FUSED_CASES = SMALL_BF16 + [
+    RoundConfig("start", H=2, D=128, fh=10, fw=12, F=2, Wc=5, R=3, noise_t=(250, 500, 750)),
+]
+
+
+def _fused_matches_unfused(cfg, rounds, first_n0=None):
+    """The fused path (wf_rope3d_append_kv + wf_chunk_causal_attn_rope from raw Q) against the
+    two-call path on the same inputs: O, LSE and the pool bit-identical every round, which also
+    shows the in-kernel Q' equals wf_rope3d_append's bit for bit (the MMAs are deterministic)."""
+    a = Rollout(cfg, first_n0=first_n0)
+    b = Rollout(cfg, first_n0=first_n0, fused_q_rope=True)
+    a.prefill()
+    b.prefill()
+    for r in range(rounds):
+        a.run_round(r)
+        b.run_round(r)
+        torch.cuda.synchronize()
+        assert torch.equal(a.out, b.out), f"{cfg.name} round {r}: O"
+        assert torch.equal(a.lse, b.lse), f"{cfg.name} round {r}: LSE"
+        assert torch.equal(a.k_pool, b.k_pool) and torch.equal(a.v_pool, b.v_pool), f"{cfg.name} round {r}: pool"
+    assert b.device_status()[0] == wf.WF_OK
+    return a, b
+
+
+@pytest.mark.parametrize("cfg", FUSED_CASES, ids=lambda c: c.name)
+def test_fused_q_rope_bit_identical_to_two_call_path(cfg):
+    first = 1 if cfg.name == "start" else None
+    _fused_matches_unfused(cfg, cfg.Wc + cfg.R + 2, first_n0=first)
+
+
+def test_fused_q_rope_full_size_round_against_oracle():
+    cfg = CONFIGS["wan13b_round"]
+    a, b = _fused_matches_unfused(cfg, 2)
+    rows = gc.sample_rows(cfg, extra=8)
+    gc.check_attention(b, 1, [4], rows, "fused wan13b r1")
