@@ -416,12 +416,7 @@ __device__ __forceinline__ void rope_q_role(const Shared& sh, const Params& p, i
     }
     // make the rotated tile visible to the tensor cores (async proxy)
     fence_proxy_async_smem();
-#if WF_WARP_ARRIVE
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(sh.bars + L::kQFull + buf));
-#else
     mbar_arrive(smem_u32(sh.bars + L::kQFull + buf));
-#endif
   }
 }
 
@@ -559,20 +554,6 @@ __device__ __forceinline__ void mma_issuer(const Shared& sh, const Params& p, ui
   }
 }
 
-// Softmax variants under measurement (0 = off).
-#ifndef WF_SPLIT_LD
-#define WF_SPLIT_LD 0
-#endif
-#ifndef WF_WARP_ARRIVE
-#define WF_WARP_ARRIVE 0
-#endif
-#ifndef WF_WIDE_MAX
-#define WF_WIDE_MAX 0
-#endif
-#ifndef WF_LANE0_WAIT
-#define WF_LANE0_WAIT 0
-#endif
-
 // exp2 of one row's 128 scores (scaled by sl2, minus the reference max m_ref)
 // stored as bf16 pairs into TMEM at s_tm; returns the row sum of the fp32
 // values.  Every exp2 runs on MUFU (masked columns hold -inf and give +0).
@@ -640,63 +621,11 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
         key_tile(c, j, tok, valid);
       }
       // warp-uniform: the TMEM loads and stores below are warp-collective
-#if WF_LANE0_WAIT
-      {
-        // one lane polls the barrier; the warp synchronises on its result
-        bool okw = true;
-        if (lane == 0) okw = wait_bar(sh, p, L::kSFull + t, s_cnt & 1, 20 + t);
-        __syncwarp();
-        if (!__shfl_sync(0xffffffffu, okw, 0)) return;
-      }
-#else
       if (!__all_sync(0xffffffffu, wait_bar(sh, p, L::kSFull + t, s_cnt & 1, 20 + t))) return;
-#endif
       ++s_cnt;
       tc_fence_after();
       float s[128];
       float mxs[8];
-#if WF_SPLIT_LD
-      // two halves: the second half's TMEM load is in flight while the
-      // first half's columns are reduced
-#pragma unroll
-      for (int q4 = 0; q4 < 2; ++q4) {
-        uint32_t r[32];
-        tmem_ld32(s_tm + 32 * q4, r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[32 * q4 + x] = __uint_as_float(r[x]);
-      }
-      tmem_wait_ld();
-#pragma unroll
-      for (int q4 = 2; q4 < 4; ++q4) {
-        uint32_t r[32];
-        tmem_ld32(s_tm + 32 * q4, r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[32 * q4 + x] = __uint_as_float(r[x]);
-      }
-      if (valid < 64) {
-#pragma unroll
-        for (int x = 0; x < 64; ++x)
-          if (x >= valid) s[x] = -INFINITY;
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(s[c], s[c + 8]);
-#pragma unroll
-      for (int x = 16; x < 64; x += 16) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
-      }
-      tmem_wait_ld();
-      if (valid < 128) {
-#pragma unroll
-        for (int x = 64; x < 128; ++x)
-          if (x >= valid) s[x] = -INFINITY;
-      }
-#pragma unroll
-      for (int x = 64; x < 128; x += 16) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
-      }
-#else
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t r[32];
@@ -710,17 +639,6 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
         for (int x = 0; x < 128; ++x)
           if (x >= valid) s[x] = -INFINITY;
       }
-#if WF_WIDE_MAX
-      // a shallower reduction: 32 three-input maxima over disjoint quadruples
-      // (depth 2), then a tree (depth 4) -- 6 dependent steps instead of 11
-      {
-        float m32[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) m32[c] = max3f(s[4 * c], s[4 * c + 1], fmaxf(s[4 * c + 2], s[4 * c + 3]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(max3f(m32[c], m32[c + 8], m32[c + 16]), m32[c + 24]);
-      }
-#else
 #pragma unroll
       for (int c = 0; c < 8; ++c) mxs[c] = fmaxf(s[c], s[c + 8]);
 #pragma unroll
@@ -728,8 +646,6 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
 #pragma unroll
         for (int c = 0; c < 8; ++c) mxs[c] = max3f(mxs[c], s[x + c], s[x + 8 + c]);
       }
-#endif
-#endif
       const float mx = fmaxf(max3f(mxs[0], mxs[1], mxs[2]), max3f(mxs[3], max3f(mxs[4], mxs[5], mxs[6]), mxs[7]));
       const float m_new = fmaxf(m_ref, mx * sl2);
       if (j == t0) {
@@ -758,14 +674,7 @@ __device__ __forceinline__ void softmax_role(const Shared& sh, const Params& p, 
       l += exp_to_p(s, sl2, m_ref, s_tm);
       tmem_wait_st();
       tc_fence_before();
-#if WF_WARP_ARRIVE
-      // one arrival per warp (after every lane's stores have completed): 128
-      // per-thread arrivals on one barrier took ~250 cycles to land
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(sh.bars + L::kPFull + t));
-#else
       mbar_arrive(smem_u32(sh.bars + L::kPFull + t));
-#endif
     }
     // epilogue: O / l -> bf16 rows of this tile (a part of a split unit:
     // fp32 rows and the LSE into its partial slot, merged by the combine pass)
@@ -829,8 +738,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 9 && lane == 0) {
     for (int b = 0; b < L::kNumBars; ++b) {
       uint32_t count = 1;
-      if (b == L::kPFull || b == L::kPFull + 1) count = WF_WARP_ARRIVE ? 4 : 128;  // the tile's softmax warps
-      if (kRopeQ && b >= L::kQFull && b < L::kQFull + L::kQBufs) count = WF_WARP_ARRIVE ? 2 : 64;  // rotation
+      if (b == L::kPFull || b == L::kPFull + 1) count = 128;  // the tile's softmax threads
+      if (kRopeQ && b >= L::kQFull && b < L::kQFull + L::kQBufs) count = 64;  // the rotation threads
       mbar_init(smem_u32(sh.bars + b), count);
     }
     *sh.abort_flag = 0;
