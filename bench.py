@@ -26,7 +26,9 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
+from typing import Optional
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -112,16 +114,68 @@ def replica_seed(rank: int) -> int:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled DURING the timed region.
+
+    NVML is polled in a thread every ~2 ms and each sample is timestamped, so
+    that only the samples inside [t0, t1] (host times bracketing the timed
+    region: the queue is empty at t0 and drained at t1) are summarised; a
+    timed region of ~100 ms then still yields dozens of samples.  Without
+    NVML it falls back to `nvidia-smi -lms 200` over the whole window."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvmlClocksEventReason*)
+    REASON_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                   ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
+    PERIOD_S = 0.002
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: Optional[str] = None):
         self.gpu = gpu_index
+        self.uuid = uuid
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.handle = None
+        self.rows = []
+        self.thread = None
+        self.stop_flag = False
+
+    def _open_nvml(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = None
+            if self.uuid:
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + self.uuid)
+                except Exception:  # noqa: BLE001 - fall back to the index
+                    handle = None
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.nvml, self.handle = pynvml, handle
+            return True
+        except Exception:  # noqa: BLE001 - no NVML: use nvidia-smi
+            return False
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_flag:
+            try:
+                row = (time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax,
+                       nv.nvmlDeviceGetPowerUsage(h) / 1000.0, nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.rows.append(row)
+            except Exception:  # noqa: BLE001 - a failed query skips one sample
+                pass
+            time.sleep(self.PERIOD_S)
 
     def start(self):
+        self.rows = []
+        if self._open_nvml():
+            self.stop_flag = False
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         fd, self.path = tempfile.mkstemp(prefix="wf_clocks_", suffix=".csv")
         os.close(fd)
         try:
@@ -131,7 +185,28 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self):
+    @classmethod
+    def summarise(cls, rows, t0=None, t1=None):
+        """rows: (time, sm_mhz, sm_max_mhz, power_w, reason_bits).  Summary of
+        the rows inside [t0, t1] (all rows if no window is given)."""
+        inside = [r for r in rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [r[1] for r in inside]
+        bits = 0
+        for r in inside:
+            bits |= int(r[4])
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(r[2] for r in inside),
+                "power_w_median": round(statistics.median(r[3] for r in inside), 1),
+                "reasons": sorted(n for n, bit in cls.REASON_BITS if bits & bit),
+                "samples": len(inside), "source": f"NVML every {1e3 * cls.PERIOD_S:.0f} ms inside the timed region"}
+
+    def stop(self, t0=None, t1=None):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=10)
+            self.thread = None
+            return self.summarise(self.rows, t0, t1)
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.25)
@@ -152,7 +227,7 @@ class ClockSampler:
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi every 200 ms over the whole window"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) sample
@@ -276,19 +351,24 @@ def run_wf(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]),
+                           uuid=str(getattr(props, "uuid", "") or "") or None)
     sampler.start()
-    time.sleep(0.3)
+    if sampler.thread is None:
+        time.sleep(0.3)  # nvidia-smi's first sample
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    host_t0 = time.perf_counter()
     t_start.record(stream)
     for s in range(K):
         step(W + s, ev[s])
     t_end.record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop()
+    host_t1 = time.perf_counter()
+    clocks = sampler.stop(host_t0, host_t1)
     # host time of planning one round (wf_plan_round without the device copy),
     # reported beside the device-timed step
     plan_host = torch.empty(wf.wf_plan_bytes(ro.desc(ro.n0_of(W + K))), dtype=torch.uint8)

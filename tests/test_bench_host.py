@@ -56,3 +56,18 @@ def test_reference_arm_line_has_the_contract_fields():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert bench.run_reference(Args, 1, 2) is None  # other ranks do no work
+
+
+def test_clock_summary_keeps_only_the_timed_region_and_decodes_reasons():
+    bench = _bench()
+    rows = [(0.0, 1965, 1965, 300.0, 0x1),      # idle before the region
+            (1.0, 1800, 1965, 900.0, 0x4),      # sw_power_cap
+            (1.1, 1700, 1965, 950.0, 0x4),
+            (1.2, 1650, 1965, 980.0, 0x4 | 0x40),  # plus hw_thermal_slowdown
+            (3.0, 1965, 1965, 250.0, 0x1)]      # idle after it
+    got = bench.ClockSampler.summarise(rows, 0.5, 2.0)
+    assert got["samples"] == 3
+    assert got["sm_mhz"] == 1700 and got["sm_min_mhz"] == 1650 and got["sm_max_mhz"] == 1965
+    assert got["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.ClockSampler.summarise(rows, 5.0, 6.0)["reasons"] == ["no samples"]
+    assert bench.ClockSampler.summarise(rows)["samples"] == 5
