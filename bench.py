@@ -50,6 +50,8 @@ def parse_args():
                     help="the attention rotates the raw Q itself; the append pass writes only K'/V")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8-side", action="store_true",
+                    help="skip the side measurement of the 8-bit score variant on a 16-bit run")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -302,6 +304,51 @@ def run_reference(args, rank, world):
     return line
 
 
+def fp8_side(cfg, dev, stream, rank, world, W, K):
+    """The same rounds with 8-bit (e4m3) scores, device-timed like the main
+    run (plan, RoPE/append, both quantizations, attention per step; inputs
+    drawn on the device before timing), so that one default run records both
+    variants.  Returns the summary for the JSON line."""
+    import torch
+    from chunk_causal_attention_block_b200 import wf
+    from chunk_causal_attention_block_b200.rollout import Rollout
+
+    ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank), fp8=True)
+    ro.prefill()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    # inputs are drawn per round on the device; only plan + kernels are timed
+    for r in range(W):
+        ro.fill_inputs(ro.n0_of(r), cfg.R, r)
+        ro.plan_round(r)
+        ro.append()
+        ro.attend()
+    torch.cuda.synchronize()
+    step_ms = []
+    for s in range(K):
+        r = W + s
+        ro.fill_inputs(ro.n0_of(r), cfg.R, r)
+        ev[s][0].record(stream)
+        ro.plan_round(r)
+        ro.append()
+        ev[s][1].record(stream)
+        ro.attend()
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    code, detail = ro.device_status()
+    if code != wf.WF_OK:
+        raise RuntimeError(f"device status (8-bit scores) {wf.status_string(code)} {detail}")
+    attn = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    step = statistics.mean(e[0].elapsed_time(e[2]) for e in ev)
+    attn = max_over_ranks(attn, world, dev)
+    step = max_over_ranks(step, world, dev)
+    flops = cfg.attn_flops()
+    return {"attn_tflops_kernel": flops / (attn / 1e3) / 1e12, "step_tflops": flops * world / (step / 1e3) / 1e12,
+            "attn_ms": attn, "ms_per_step": step, "steps": K, "warmup": W,
+            "dtype": "e4m3 scores, bf16 P/V/O", "gpu_launches": 4 * K,
+            "timing": "device events per step around plan+RoPE/append+quantize and attention; "
+                      "input drawing between steps is outside them"}
+
+
 def run_wf(args, rank, world, local_rank):
     import numpy as np  # noqa: F401
     import torch
@@ -319,6 +366,7 @@ def run_wf(args, rank, world, local_rank):
     ro = Rollout(cfg, device=dev, want_lse=False, seed=replica_seed(rank), fp8=args.scores == "fp8",
                  fused_q_rope=args.fused_q_rope)
     ro.prefill()
+    first_n0, n0_first = ro.first_n0, ro.n0_of(0)  # the oracle sample's round
 
     # every step's inputs resident in HBM before timing (round r draws tag r)
     tdt = torch.bfloat16 if cfg.dtype == wf.WF_BF16 else torch.float32
@@ -473,6 +521,10 @@ def run_wf(args, rank, world, local_rank):
         if code != wf.WF_OK:
             raise RuntimeError(f"device status {wf.status_string(code)} {detail}")
 
+    side = None
+    if args.scores == "bf16" and cfg.dtype == wf.WF_BF16 and not args.fused_q_rope and not args.no_fp8_side:
+        side = fp8_side(cfg, dev, stream, rank, world, W, K)
+
     if rank != 0:
         return None
     peaks, peak_kind = load_peaks()
@@ -520,8 +572,10 @@ def run_wf(args, rank, world, local_rank):
         "clocks": clocks,
         "e2e": e2e,
     }
+    if side is not None:
+        line["fp8_scores"] = side
     if world == 1 and not args.no_cpu_baseline:
-        f, t, desc = oracle_sample(cfg, args.cpu_seconds, ro.first_n0, ro.n0_of(0))
+        f, t, desc = oracle_sample(cfg, args.cpu_seconds, first_n0, n0_first)
         line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
                                 "kind": "oracle", "sample": desc, "seconds": t}
     return line
