@@ -63,3 +63,9 @@ extern "C" wf_status wf_chunk_causal_attn_noalloc(const void* host_plan, const v
   return wf_chunk_causal_attn(host_plan, dev_plan, q_rot, k_pool, v_pool, out, lse, softmax_scale, scratch, need,
                               stream);
 }
+
+extern "C" wf_status wf_attn_noalloc_status(wf_stream_t stream, int32_t* detail) {
+  void* scratch = scratch_on_current_device();
+  if (!scratch) return WF_ERR_CUDA;
+  return wf_attn_workspace_status(scratch, stream, detail);
+}

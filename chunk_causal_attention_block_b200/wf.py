@@ -32,8 +32,8 @@ WF_FP8_Q, WF_FP8_K = 0, 1
 EXPORTS = ("wf_plan_bytes", "wf_plan_round", "wf_balance_units", "wf_rope3d_append", "wf_attn_workspace_bytes",
            "wf_attn_workspace_init", "wf_attn_workspace_status", "wf_chunk_causal_attn", "wf_rope3d_append_kv",
            "wf_chunk_causal_attn_rope",
-           "wf_chunk_causal_attn_noalloc", "wf_quantize_fp8", "wf_chunk_causal_attn_fp8", "wf_status_string",
-           "wf_version", "wf_synth_fill")
+           "wf_chunk_causal_attn_noalloc", "wf_attn_noalloc_status", "wf_quantize_fp8", "wf_chunk_causal_attn_fp8",
+           "wf_status_string", "wf_version", "wf_synth_fill")
 
 
 class WfError(RuntimeError):
@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.wf_chunk_causal_attn.restype = i32
         L.wf_chunk_causal_attn_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp]
         L.wf_chunk_causal_attn_noalloc.restype = i32
+        L.wf_attn_noalloc_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        L.wf_attn_noalloc_status.restype = i32
         L.wf_quantize_fp8.argtypes, L.wf_quantize_fp8.restype = [vp, vp, vp, vp, i32, vp], i32
         L.wf_chunk_causal_attn_fp8.argtypes = [vp] * 9 + [ctypes.c_float, vp, sz, vp]
         L.wf_chunk_causal_attn_fp8.restype = i32
@@ -210,6 +212,14 @@ def wf_chunk_causal_attn_noalloc(host_plan, dev_plan, q_rot, k_pool, v_pool, out
     _check(lib().wf_chunk_causal_attn_noalloc(_ptr(host_plan), _ptr(dev_plan), _ptr(q_rot), _ptr(k_pool),
                                               _ptr(v_pool), _ptr(out), _ptr(lse), float(softmax_scale),
                                               _stream(stream)), "wf_chunk_causal_attn_noalloc")
+
+
+def wf_attn_noalloc_status(stream=None):
+    """Device status of the last no-alloc call on the current device: (status code,
+    [code, where, block, thread]); synchronises `stream`."""
+    detail = (ctypes.c_int32 * 4)()
+    code = lib().wf_attn_noalloc_status(_stream(stream), detail)
+    return code, list(detail)
 
 
 

@@ -279,8 +279,7 @@ wf_status wf_chunk_causal_attn_rope(const void* host_plan, const void* dev_plan,
  *   capture.  The call itself allocates nothing.
  * - Each call zeroes the status block on `stream` before launching.  A wait
  *   that times out is recorded there but is not returned by this call (it
- *   returns once the kernel is queued); callers that need the device status
- *   use wf_chunk_causal_attn with their own workspace.
+ *   returns once the kernel is queued); wf_attn_noalloc_status reads it.
  * - Every call shares the one array: calls that overlap on the GPU (different
  *   streams, not ordered) race on it.
  * Errors: as wf_chunk_causal_attn, plus WF_ERR_CAPACITY if the plan's
@@ -290,6 +289,19 @@ wf_status wf_chunk_causal_attn_rope(const void* host_plan, const void* dev_plan,
 wf_status wf_chunk_causal_attn_noalloc(const void* host_plan, const void* dev_plan,
                                        const void* q_rot, const void* k_pool, const void* v_pool,
                                        void* out, float* lse, float softmax_scale, wf_stream_t stream);
+
+/*
+ * wf_attn_noalloc_status -- the device status of the last
+ * wf_chunk_causal_attn_noalloc call on the current device, read from the
+ * library's static status block as wf_attn_workspace_status reads a
+ * workspace: synchronises `stream` (the stream of that call), then returns
+ * WF_OK or the error a kernel recorded (WF_ERR_DEVICE_TIMEOUT); `detail`, when
+ * non-NULL, receives 4 int32 (code, where, block, thread).  Before any
+ * no-alloc call on the device the block is all zero (WF_OK).
+ * Errors: WF_ERR_CUDA if the synchronisation, the address look-up or the copy
+ * fails.
+ */
+wf_status wf_attn_noalloc_status(wf_stream_t stream, int32_t* detail);
 
 /*
  * 8-bit scores.  The Wave Forcing abstract (arXiv 2611.00859v1) measures its

@@ -45,6 +45,7 @@ def test_noalloc_entry_point_is_bit_identical_to_regular_entry_point():
             torch.cuda.synchronize()
             assert torch.equal(ro.out, want), f"round {r} no-alloc call {call}: O differs"
             assert torch.equal(ro.lse, want_lse), f"round {r} no-alloc call {call}: LSE differs"
+            assert wf.wf_attn_noalloc_status(ro.stream) == (wf.WF_OK, [0, 0, 0, 0]), "no-alloc device status"
         # ... and the regular call again after the no-alloc calls, on the same plan
         ro.out.fill_(float("nan"))
         ro.lse.fill_(float("nan"))
