@@ -42,7 +42,8 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=("wf", "reference"), default="wf")
+    ap.add_argument("--impl", choices=("wf", "reference", "library"), default="wf",
+                    help="library: context only -- library Blackwell attention kernels on the same work")
     ap.add_argument("--config", default="wan13b_round")
     ap.add_argument("--scores", choices=("bf16", "fp8"), default="bf16",
                     help="fp8: e4m3 Q/K codes with block scales (quantization timed with RoPE/append)")
@@ -593,11 +594,108 @@ def run_wf(args, rank, world, local_rank):
     return line
 
 
+def run_library(args, rank):
+    """Context arm, never the product path: the round's attention work (each
+    in-round chunk's queries against its visible keys, no mask inside,
+    bf16) run through two library Blackwell attention kernels from
+    flashinfer -- the TRT-LLM-gen context kernel (paged K/V) and the CuTe-DSL
+    prefill kernel -- device-timed like the main arm, on rank 0 only."""
+    if rank != 0:
+        return None
+    import torch
+    from chunk_causal_attention_block_b200.rollout import CONFIGS
+    cfg = CONFIGS[args.config]
+    line = {"impl": "library", "metric": METRIC, "unit": "TFLOP/s", "config": {"workload": cfg.name},
+            "note": "context only: library kernels on the same work, not this library's path"}
+    if not torch.cuda.is_available():
+        line["unavailable"] = "no CUDA device"
+        return line
+    try:
+        import flashinfer  # noqa: F401
+    except Exception as e:  # noqa: BLE001 - report and stop
+        line["unavailable"] = f"flashinfer not importable: {e!r}"[:200]
+        return line
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    H, D, C = cfg.H, cfg.D, cfg.C
+    kv = [int(x) for x in cfg.visible_keys()]
+    nq, nk = cfg.R * C, sum(kv)
+    flops = cfg.attn_flops()
+    g = torch.Generator(device=dev)
+    g.manual_seed(42)
+    q = torch.randn(nq, H, D, device=dev, dtype=torch.bfloat16, generator=g)
+    qo = torch.tensor([i * C for i in range(cfg.R + 1)], dtype=torch.int32, device=dev)
+    kvp = torch.tensor([0] + [sum(kv[:i + 1]) for i in range(len(kv))], dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    W, K = args.warmup, args.steps
+    stream = torch.cuda.current_stream(dev)
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "") or None
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        sampler = ClockSampler(0, uuid=uuid)
+        sampler.start()
+        t0 = time.perf_counter()
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop(t0, time.perf_counter())
+        ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+        return {"attn_tflops_kernel": flops / (ms / 1e3) / 1e12, "attn_ms": ms, "clocks": clocks}
+
+    kernels = {}
+    try:
+        from flashinfer.prefill import trtllm_batch_context_with_kv_cache
+        page = 64
+        pages = [(x + page - 1) // page for x in kv]
+        kc = torch.randn(sum(pages), H, page, D, device=dev, dtype=torch.bfloat16, generator=g)
+        vc = torch.randn(sum(pages), H, page, D, device=dev, dtype=torch.bfloat16, generator=g)
+        bt = torch.zeros(len(kv), max(pages), dtype=torch.int32, device=dev)
+        off = 0
+        for i, n in enumerate(pages):
+            bt[i, :n] = torch.arange(off, off + n, dtype=torch.int32, device=dev)
+            off += n
+        lens = torch.tensor(kv, dtype=torch.int32, device=dev)
+        ws = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+        out = torch.empty(nq, H, D, device=dev, dtype=torch.bfloat16)
+        kernels["trtllm_gen_context"] = timed(lambda: trtllm_batch_context_with_kv_cache(
+            q, (kc, vc), ws, bt, lens, C, max(kv), scale, 1.0, len(kv), qo, kvp, out=out, kv_layout="HND",
+            causal=False))
+        kernels["trtllm_gen_context"]["layout"] = f"paged K/V, HND, page {page}"
+        del kc, vc, ws
+    except Exception as e:  # noqa: BLE001 - a kernel the installed library lacks is reported, not fatal
+        kernels["trtllm_gen_context"] = {"unavailable": repr(e)[:200]}
+    try:
+        from flashinfer.cute_dsl.attention.wrappers.batch_prefill import BatchPrefillCuteDSLWrapper
+        k = torch.randn(nk, H, D, device=dev, dtype=torch.bfloat16, generator=g)
+        v = torch.randn(nk, H, D, device=dev, dtype=torch.bfloat16, generator=g)
+        w = BatchPrefillCuteDSLWrapper(torch.empty(16 << 20, dtype=torch.uint8, device=dev))
+        w.plan(qo, kvp, H, H, D, causal=False, sm_scale=scale, q_data_type=torch.bfloat16,
+               kv_data_type=torch.bfloat16)
+        o2 = torch.empty(nq, H, D, device=dev, dtype=torch.bfloat16)
+        kernels["cute_dsl_prefill"] = timed(lambda: w.run(q, k, v, out=o2))
+        kernels["cute_dsl_prefill"]["note"] = "run() includes its copy of O into the caller's tensor"
+    except Exception as e:  # noqa: BLE001
+        kernels["cute_dsl_prefill"] = {"unavailable": repr(e)[:200]}
+    line.update({"steps": K, "warmup": W, "kernels": kernels})
+    return line
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "library":
+        line = run_library(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
     if args.impl == "reference":
         # the oracle arm is CPU-only; under torchrun only rank 0 works
         line = run_reference(args, rank, world)

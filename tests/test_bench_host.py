@@ -71,3 +71,19 @@ def test_clock_summary_keeps_only_the_timed_region_and_decodes_reasons():
     assert got["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     assert bench.ClockSampler.summarise(rows, 5.0, 6.0)["reasons"] == ["no samples"]
     assert bench.ClockSampler.summarise(rows)["samples"] == 5
+
+
+def test_library_context_arm_reports_unavailable_without_a_gpu():
+    import json
+    import subprocess
+    import sys
+
+    import torch
+    if torch.cuda.is_available():
+        import pytest
+        pytest.skip("a GPU is present: the arm would run the library kernels")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "library"], capture_output=True,
+                       text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "library" and line["unavailable"] == "no CUDA device"
