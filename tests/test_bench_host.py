@@ -87,3 +87,41 @@ def test_library_context_arm_reports_unavailable_without_a_gpu():
     assert r.returncode == 0, r.stderr
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "library" and line["unavailable"] == "no CUDA device"
+
+
+def test_clock_sampler_polls_nvml_inside_the_window(monkeypatch):
+    """The sampler's NVML path against a fake NVML: samples are taken while it
+    runs, only those inside the window are kept, reasons are decoded."""
+    import sys
+    import time
+    import types
+
+    calls = {"uuid": None}
+    fake = types.ModuleType("pynvml")
+    fake.NVML_CLOCK_SM = 1
+    fake.nvmlInit = lambda: None
+
+    def by_uuid(u):
+        calls["uuid"] = u
+        return "handle"
+    fake.nvmlDeviceGetHandleByUUID = by_uuid
+    fake.nvmlDeviceGetHandleByIndex = lambda i: "handle"
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    fake.nvmlDeviceGetClockInfo = lambda h, c: 1605
+    fake.nvmlDeviceGetPowerUsage = lambda h: 985000  # mW
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4  # sw_power_cap
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    bench = _bench()
+    s = bench.ClockSampler(0, uuid="0123-abcd")
+    s.start()
+    assert s.thread is not None, "NVML path not taken"
+    time.sleep(0.02)
+    t0 = time.perf_counter()
+    time.sleep(0.05)
+    t1 = time.perf_counter()
+    time.sleep(0.02)
+    got = s.stop(t0, t1)
+    assert calls["uuid"] == "GPU-0123-abcd"
+    assert got["samples"] >= 3 and got["sm_mhz"] == 1605 and got["sm_max_mhz"] == 1965
+    assert got["power_w_median"] == 985.0 and got["reasons"] == ["sw_power_cap"]
+    assert len(s.rows) > got["samples"]  # samples outside the window were taken and dropped
