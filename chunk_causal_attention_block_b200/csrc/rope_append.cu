@@ -9,7 +9,10 @@
 // fully coalesced 512-byte run.  Index decoding uses exact multiply-shift
 // reciprocals instead of integer division.  The rotation runs in fp64 from
 // the plan's fp64 cos/sin tables (L1-resident, a few KB) and is rounded once
-// to the storage type (rope_math.cuh).
+// to the storage type (rope_math.cuh): for bf16 by the direct fp64 -> bf16
+// conversion, one conversion per element instead of the two of an fp64 ->
+// fp32 round-to-odd step and its exactness test (58.5-60 against 60.6-63 us
+// on the 4-chunk round; the conversion pipe was the kernel's limit).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -90,12 +93,12 @@ __device__ __forceinline__ void rope_vector(const RopeParams& p, uint32_t e, con
 constexpr int kRopeThreads = 256;
 
 // One 16-byte vector of each tensor per thread, a block per 256 vectors
-// (61 registers: four blocks per SM).  Measured slower on the 4-chunk round (72 us
-// for this kernel): a grid-stride loop that keeps 3-5 further steps' loads in
-// flight through cp.async into shared memory (85-98 us), half vectors per
-// thread at 6 or 8 blocks per SM (82 us, issue-bound at 75% issue activity),
-// and converting bf16 -> fp64 or testing the round-to-odd exactness with
-// integer operations instead of conversions (83-91 us).
+// (62 registers: four blocks per SM).  Measured slower on the 4-chunk round,
+// against 72 us for the kernel of the time: a grid-stride loop that keeps 3-5
+// further steps' loads in flight through cp.async into shared memory (85-98
+// us), half vectors per thread at 6 or 8 blocks per SM (82 us, issue-bound at
+// 75% issue activity), and converting bf16 -> fp64 or testing a round-to-odd
+// step's exactness with integer operations instead of conversions (83-91 us).
 template <typename T, bool kWithQ>
 __global__ void __launch_bounds__(kRopeThreads)
     rope3d_append_kernel(RopeParams p, const uint4* __restrict__ q, const uint4* __restrict__ k,

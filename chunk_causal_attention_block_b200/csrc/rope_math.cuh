@@ -27,17 +27,9 @@ __device__ __forceinline__ double2 rope_cos_sin(const double2* tab_t, const doub
   return __ldg(e);
 }
 
-// x rounded toward zero to fp32 with the last bit set when that lost anything
-// ("round to odd"); rounding that to bf16 to nearest-even then equals direct
-// nearest-even rounding of x (Boldo and Melquiond, "Emulation of FMA and
-// correctly rounded sums: proved algorithms using rounding to odd", IEEE TC
-// 2008: rounding to odd in a format with at least two more bits makes the
-// second rounding correct).
-__device__ __forceinline__ float f64_to_f32_round_odd(double x) {
-  float r = __double2float_rz(x);
-  if (double(r) != x) r = __int_as_float(__float_as_int(r) | 1);
-  return r;
-}
+// x rounded once, to nearest even, to bf16: the conversion instruction rounds
+// from fp64 directly (cvt.rn.bf16.f64).
+__device__ __forceinline__ uint16_t f64_to_bf16_bits(double x) { return __bfloat16_as_ushort(__double2bfloat16(x)); }
 
 __device__ __forceinline__ void rotate_pair(double x, double y, double2 cs, double& xr, double& yr) {
   // same operation order as a plain fp64 evaluation of x*c - y*s, x*s + y*c
@@ -62,10 +54,10 @@ struct Pack<__nv_bfloat16> {
   }
   __device__ static uint4 pack(const double* in) {
     uint4 v;
-    __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&v);
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      p[i] = __floats2bfloat162_rn(f64_to_f32_round_odd(in[2 * i]), f64_to_f32_round_odd(in[2 * i + 1]));
+      w[i] = uint32_t(f64_to_bf16_bits(in[2 * i])) | (uint32_t(f64_to_bf16_bits(in[2 * i + 1])) << 16);
     return v;
   }
 };
@@ -93,8 +85,7 @@ __device__ __forceinline__ uint32_t rope_pair_bf16(uint32_t word, double2 cs) {
   const float2 xy = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&word));
   double xr, yr;
   rotate_pair(double(xy.x), double(xy.y), cs, xr, yr);
-  const __nv_bfloat162 r = __floats2bfloat162_rn(f64_to_f32_round_odd(xr), f64_to_f32_round_odd(yr));
-  return *reinterpret_cast<const uint32_t*>(&r);
+  return uint32_t(f64_to_bf16_bits(xr)) | (uint32_t(f64_to_bf16_bits(yr)) << 16);
 }
 
 }  // namespace
