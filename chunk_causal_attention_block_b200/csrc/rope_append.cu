@@ -11,8 +11,8 @@
 // the plan's fp64 cos/sin tables (L1-resident, a few KB) and is rounded once
 // to the storage type (rope_math.cuh): for bf16 by the direct fp64 -> bf16
 // conversion, one conversion per element instead of the two of an fp64 ->
-// fp32 round-to-odd step and its exactness test (58.5-60 against 60.6-63 us
-// on the 4-chunk round; the conversion pipe was the kernel's limit).
+// fp32 round-to-odd step and its exactness test (57.9 against 62.0 us for
+// the 4-chunk round's launch under ncu; the conversion pipe was the limit).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
